@@ -1,0 +1,365 @@
+"""Benchmark of the streamed decoder-stack training step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+A step is one call of ``mt_stream_step``: forward over the whole stack with
+checkpoints every K layers, then per segment re-forward, recompute and
+backward, with every layer's bf16 weights streamed in from the pinned host
+store and its fp32 gradients streamed out through the slab pool. Workloads
+(synthetic data, seeded, N(0, 0.02) weights, N(0, 1) inputs and dY):
+
+  1 tiny      hidden 256, 4/2 heads x 64, FFN 688, 1 layer, batch 2 x 128
+  2 7b_x4     Qwen2.5-7B layer shape x 4 layers, batch 8 x 1024, K = 4  (default)
+  3 7b_x28    7B shape x 28 layers, batch 96 x 1024, K = 4
+  4 14b_x48   Qwen2.5-14B shape x 48 layers, batch 64 x 1024, K = 4
+  5 7b_32k    7B shape x 28 layers, batch 1 x 32768, MLP in 4096-token chunks, K = 4
+
+The metric is sustained TFLOPS by the model-FLOPs formula 6ND + 12LHT^2
+(MegaTrain Table 7 caption) with N = layers x parameters per layer, plus
+tokens/s. One process per GPU; with N > 1 (torchrun) every rank runs its own
+replica on its own batch (the path has no collective), the timed region is
+bracketed by barriers and the slowest rank's time is used.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on a bounded
+sample of the same workload and reports the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from host_offloaded_layer_b200 import metrics, synth  # noqa: E402
+
+QWEN7B = dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944)
+QWEN14B = dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824)
+CONFIGS = {
+    1: dict(name="tiny_1layer_b2x128", shape=dict(hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=688),
+            L=1, B=2, T=128, K=4, chunk=0),
+    2: dict(name="qwen2.5-7b-shape_x4_b8x1024", shape=QWEN7B, L=4, B=8, T=1024, K=4, chunk=0),
+    3: dict(name="qwen2.5-7b-shape_x28_b96x1024", shape=QWEN7B, L=28, B=96, T=1024, K=4, chunk=0),
+    4: dict(name="qwen2.5-14b-shape_x48_b64x1024", shape=QWEN14B, L=48, B=64, T=1024, K=4, chunk=0),
+    5: dict(name="qwen2.5-7b-shape_x28_b1x32768_mlpchunk4096", shape=QWEN7B, L=28, B=1, T=32768, K=4, chunk=4096),
+}
+METRIC = "sustained TFLOPS (6ND+12LHT²) & tokens/s, streamed 7B/14B layer stack, 1 B200"
+UNIT = "TFLOPS"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def model_flops(cfg, p_layer):
+    sh = cfg["shape"]
+    return metrics.model_flops(cfg["L"] * p_layer, cfg["L"], sh["hidden"], cfg["B"], cfg["T"])
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- host link
+def measure_link(torch, nbytes=1 << 30):
+    """Pinned-memory copy bandwidth (GB/s): H2D, D2H, and both at once."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h2 = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d2 = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def timed(fn, reps=3):
+        best = 1e9
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            best = min(best, time.perf_counter() - t0)
+        return best
+
+    with torch.cuda.stream(s1):
+        t_h2d = timed(lambda: d.copy_(h, non_blocking=True))
+        t_d2h = timed(lambda: h.copy_(d, non_blocking=True))
+
+    def both():
+        with torch.cuda.stream(s1):
+            d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h2.copy_(d2, non_blocking=True)
+
+    t_both = timed(both)
+    del h, h2, d, d2
+    return {"h2d_gbs": nbytes / t_h2d / 1e9, "d2h_gbs": nbytes / t_d2h / 1e9, "bidir_gbs": 2 * nbytes / t_both / 1e9}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(cfg, budget_s=12.0):
+    """Times the float64 oracle (forward + backward of one layer of this
+    workload's shape) on a bounded token sample; returns (TFLOPS, desc, threads)."""
+    from oracle import OracleCfg, layer_bwd, layer_fwd
+    sh = cfg["shape"]
+    T = min(cfg["T"], 256)
+    B = 1
+    ocfg = OracleCfg(**sh)
+    shapes = synth.layer_tensor_shapes(**sh)
+    w = {k: synth.bf16_round(v).astype(np.float64) for k, v in synth.layer_weights_f32(shapes, 1234, 0).items()}
+    x = synth.bf16_bits_to_f32(synth.activations_bf16_bits(1234, synth.X0_ID, B, T, sh["hidden"])).astype(np.float64)
+    dy = synth.bf16_bits_to_f32(synth.activations_bf16_bits(1234, synth.DY_ID, B, T, sh["hidden"])).astype(np.float64)
+    p_layer = sum(int(np.prod(s)) for s in shapes.values())
+    flops = metrics.model_flops(p_layer, 1, sh["hidden"], B, T)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        y, cache = layer_fwd(ocfg, w, x)
+        layer_bwd(ocfg, w, cache, dy)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    threads = os.environ.get("OPENBLAS_NUM_THREADS") or os.environ.get("OMP_NUM_THREADS") or str(os.cpu_count())
+    desc = f"1 layer of the workload's shape, forward+backward, batch {B} x {T} tokens, {reps} reps in {el:.1f} s"
+    return flops * reps / el / 1e12, desc, int(threads), el / reps
+
+
+def run_reference(args, cfg, rank, world):
+    """The reference arm: the CPU oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, desc, threads, sec = oracle_sample(cfg, budget_s=max(1.0, 20.0 / max(1, args.steps + args.warmup)))
+        if i >= args.warmup:
+            vals.append(tf)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg["name"], "sample": desc},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- ours
+def fill_store(L_, store, cfg, n_layers, seed=1234):
+    off = L_.mt_layer_param_offsets(cfg)
+    shapes = synth.layer_tensor_shapes(cfg.hidden, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn,
+                                       bool(cfg.qkv_bias))
+    for l in range(n_layers):
+        ptr = L_.mt_host_store_master(store, l)
+        master = np.ctypeslib.as_array((ctypes.c_float * off.record_elems).from_address(ptr))
+        for name, shp in shapes.items():
+            o = getattr(off, name)
+            n = int(np.prod(shp))
+            if name in ("g1", "g2"):
+                master[o:o + n] = 1.0
+            else:
+                synth.normal_f32(seed, l, synth.TENSOR_IDS[name], n, synth.WEIGHT_STD, out=master[o:o + n])
+    L_.mt_host_store_refresh_bf16(store, 0)
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    from host_offloaded_layer_b200 import _lib as L_
+    torch.cuda.set_device(local_rank)
+    L_.load()
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    sh = cfg["shape"]
+    lcfg = L_.make_cfg(**sh)
+    p_layer = L_.mt_layer_param_count(lcfg)
+    nL, B, T = cfg["L"], cfg["B"], cfg["T"]
+    opts = L_.make_opts(ckpt_interval=cfg["K"], mlp_chunk=cfg["chunk"], time_gemms=1, timeout_ms=120000)
+    store = L_.mt_host_store_create(lcfg, nL, True)
+    fill_store(L_, store, lcfg, nL)
+    nbytes = L_.mt_engine_workspace_bytes(lcfg, nL, B, T, opts)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    eng = L_.mt_engine_create(lcfg, nL, B, T, opts, ws, nbytes, *streams)
+    H = sh["hidden"]
+    x0 = synth.activations_bf16_bits(1234 + rank, synth.X0_ID, B, T, H)
+    dy = synth.activations_bf16_bits(1234 + rank, synth.DY_ID, B, T, H)
+    x_d = torch.from_numpy(x0.view(np.int16)).cuda()
+    dy_d = torch.from_numpy(dy.view(np.int16)).cuda()
+    y_d, dx_d = torch.empty_like(x_d), torch.empty_like(x_d)
+    xh, dyh = torch.from_numpy(x0.view(np.int16)).pin_memory(), torch.from_numpy(dy.view(np.int16)).pin_memory()
+    yh, dxh = torch.empty_like(xh).pin_memory(), torch.empty_like(xh).pin_memory()
+    slab_count = [0]
+
+    def sink(layer, ptr, n, user):  # the gradient record of one layer arrives in host memory
+        slab_count[0] += 1
+        return 0
+
+    c_sink = L_.mt_grad_sink(sink)
+    cs = streams[0]
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        barrier()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(cs)
+        for _ in range(steps):
+            fn()
+        ev1.record(cs)
+        barrier()
+        ms = ev0.elapsed_time(ev1)
+        if pg is not None:
+            t = torch.tensor([ms], device="cuda")
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms / steps
+
+    dev_step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d, c_sink)  # noqa: E731
+    host_step = lambda: L_.mt_stream_step_host(eng, store, xh, dyh, yh, dxh, c_sink)  # noqa: E731
+    for _ in range(args.warmup):
+        dev_step()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ms = timed(dev_step, args.steps)
+    clk = clocks.stop()
+    st = L_.mt_engine_stats(eng)  # the last timed step
+    for _ in range(1):
+        host_step()
+    ms_e2e = timed(host_step, max(1, args.steps // 2))
+    st_e2e = L_.mt_engine_stats(eng)
+    assert L_.mt_device_error(clear=True) == 0, "a kernel's bounded wait ran out"
+    link = measure_link(torch) if rank == 0 else None
+
+    mflops = model_flops(cfg, p_layer)
+    value = mflops * world / (ms / 1e3) / 1e12
+    e2e = mflops * world / (ms_e2e / 1e3) / 1e12
+    peaks, src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    gemm_tf = st.gemm_flops / (st.gemm_ms / 1e3) / 1e12 if st.gemm_ms > 0 else None
+    line = None
+    if rank == 0:
+        bw = link
+        t_comp = st.exec_flops / (peak_tf * 1e12)
+        t_h2d = st.h2d_bytes / (bw["h2d_gbs"] * 1e9)
+        t_d2h = st.d2h_bytes / (bw["d2h_gbs"] * 1e9)
+        t_bi = (st.h2d_bytes + st.d2h_bytes) / (bw["bidir_gbs"] * 1e9)
+        t_roof = max(t_comp, t_h2d, t_d2h, t_bi)
+        cpu_tf, cpu_desc, cpu_threads, _ = oracle_sample(cfg, budget_s=12.0)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg["name"], "layers": nL, "batch": B, "seq_len": T, "ckpt_interval": cfg["K"],
+                       "mlp_chunk": cfg["chunk"], "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (each layer's weights alone are %.0f MB)" % (p_layer * 2 / 1e6),
+                       "sink": "pinned slab handed to a no-op host callback"},
+            "tokens_per_s": B * T * world / (ms / 1e3),
+            "clocks": clk,
+            "e2e": {"value": e2e, "unit": UNIT,
+                    "h2d_bytes_per_step": int(st_e2e.h2d_bytes), "d2h_bytes_per_step": int(st_e2e.d2h_bytes)},
+            "gpu_launches": int(st.kernel_launches) * args.steps,
+            "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05)", "achieved": gemm_tf,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": (gemm_tf / peak_tf) if gemm_tf else None,
+                         "traffic": None, "peak_source": f"{src} bf16_tflops_sustained",
+                         "gemm_launches_per_step": int(st.gemm_launches)},
+            "step_roofline": {"t_roof_ms": t_roof * 1e3, "t_step_ms": ms, "frac": t_roof / (ms / 1e3),
+                              "t_compute_ms": t_comp * 1e3, "t_h2d_ms": t_h2d * 1e3, "t_d2h_ms": t_d2h * 1e3,
+                              "t_bidir_ms": t_bi * 1e3, "exec_tflop": st.exec_flops / 1e12,
+                              "model_tflop": mflops / 1e12, "h2d_bytes": int(st.h2d_bytes),
+                              "d2h_bytes": int(st.d2h_bytes), "link_gbs": bw,
+                              "model_flops_frac": mflops / (ms / 1e3) / (peak_tf * 1e12)},
+            "cpu_baseline": {"value": cpu_tf, "unit": UNIT, "cores": cpu_threads, "kind": "oracle",
+                             "sample": cpu_desc},
+            "device_workspace_gb": nbytes / 1e9,
+        }
+    L_.mt_engine_destroy(eng)
+    L_.mt_host_store_destroy(store)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    rank, world, local_rank = dist_env()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+    else:
+        run_ours(args, cfg, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,684 @@
+// Host store and streaming engine.
+//
+// The MegaTrain pages describe a memory-centric executor: parameters live in
+// host memory (abstract; Fig. 2; blog design point 1) in a flat layout that
+// keeps host memory linear in the parameter count (blog, Performance), and
+// each training step streams a layer's weights in and its gradients out
+// (blog design point 2) through a pipelined, double-buffered engine on three
+// CUDA streams - weight prefetch (W), compute (F/R/B) and gradient offload
+// (G) - so that transfers stay off the critical path (abstract; Fig. 3).
+// Activations are checkpointed every K layers and recomputed (blog design
+// point 3), and gradients pass through a pool of recycled pinned slabs
+// (Table 4, "Gradient Slab Pool").
+//
+// Here one host thread enqueues every copy and kernel of a step ahead of the
+// GPU, ordered only by CUDA events:
+//   prefetch: wait done[prev user of slot] -> H2D record -> record ready
+//   compute : wait ready -> layer template -> record done (and g_ready)
+//   offload : wait g_ready -> D2H into a pooled pinned slab -> record d2h_done
+// A second host thread polls d2h_done (bounded), hands each slab to the sink
+// in backward order and returns it to the pool. Every host wait is bounded by
+// the engine's timeout; nothing waits on the device.
+#include <atomic>
+#include <chrono>
+#include <condition_variable>
+#include <cstring>
+#include <deque>
+#include <functional>
+#include <mutex>
+#include <thread>
+#include <vector>
+
+#include "mt_internal.h"
+
+namespace mt {
+struct Use {
+  int32_t layer, kind;
+};
+std::vector<Use> build_uses(int L, int K);
+void plan_slots(const std::vector<Use>& u, int R, std::vector<int>& slot, std::vector<int>& load);
+}  // namespace mt
+
+using namespace mt;
+
+// ======================================================================= host store
+struct mt_host_store {
+  Geom G;
+  int L;
+  float* master = nullptr;
+  uint16_t* bf = nullptr;
+};
+
+static void parallel_for(int64_t n, int threads, const std::function<void(int64_t, int64_t)>& fn) {
+  if (threads <= 1 || n < (1 << 20)) {
+    fn(0, n);
+    return;
+  }
+  std::vector<std::thread> th;
+  const int64_t per = (n + threads - 1) / threads;
+  for (int t = 0; t < threads; ++t) {
+    const int64_t a = t * per, b = std::min(n, a + per);
+    if (a >= b) break;
+    th.emplace_back([&fn, a, b] { fn(a, b); });
+  }
+  for (auto& x : th) x.join();
+}
+
+static int default_threads() {
+  unsigned n = std::thread::hardware_concurrency();
+  return n == 0 ? 4 : static_cast<int>(std::min(n, 32u));
+}
+
+extern "C" {
+
+mt_status mt_host_store_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t keep_fp32_master,
+                               mt_host_store** out) {
+  if (!out) return fail(MT_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  Geom G;
+  MT_TRY(make_geom(cfg, &G));
+  if (n_layers <= 0) return fail(MT_ERR_INVALID_ARG, "n_layers must be positive");
+  auto* s = new mt_host_store();
+  s->G = G;
+  s->L = n_layers;
+  const uint64_t n = G.off.record_elems * static_cast<uint64_t>(n_layers);
+  if (cudaHostAlloc(reinterpret_cast<void**>(&s->bf), n * 2, cudaHostAllocPortable) != cudaSuccess) {
+    cudaGetLastError();
+    delete s;
+    return fail(MT_ERR_OOM, "pinned allocation of %llu bytes (bf16 store) failed", (unsigned long long)(n * 2));
+  }
+  if (keep_fp32_master) {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->master), n * 4, cudaHostAllocPortable) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFreeHost(s->bf);
+      delete s;
+      return fail(MT_ERR_OOM, "pinned allocation of %llu bytes (fp32 master) failed", (unsigned long long)(n * 4));
+    }
+  }
+  parallel_for(static_cast<int64_t>(n), default_threads(), [s](int64_t a, int64_t b) {
+    std::memset(s->bf + a, 0, (b - a) * 2);
+    if (s->master) std::memset(s->master + a, 0, (b - a) * 4);
+  });
+  *out = s;
+  return MT_OK;
+}
+
+float* mt_host_store_master(mt_host_store* s, int32_t layer) {
+  if (!s || !s->master || layer < 0 || layer >= s->L) return nullptr;
+  return s->master + static_cast<uint64_t>(layer) * s->G.off.record_elems;
+}
+
+mt_bf16* mt_host_store_bf16(mt_host_store* s, int32_t layer) {
+  if (!s || layer < 0 || layer >= s->L) return nullptr;
+  return s->bf + static_cast<uint64_t>(layer) * s->G.off.record_elems;
+}
+
+mt_status mt_host_store_refresh_bf16(mt_host_store* s, int32_t n_threads) {
+  if (!s) return fail(MT_ERR_INVALID_ARG, "store is NULL");
+  if (!s->master) return fail(MT_ERR_INVALID_ARG, "store has no fp32 master copy");
+  const int64_t n = static_cast<int64_t>(s->G.off.record_elems) * s->L;
+  parallel_for(n, n_threads > 0 ? n_threads : default_threads(), [s](int64_t a, int64_t b) {
+    for (int64_t i = a; i < b; ++i) {
+      uint32_t u;
+      std::memcpy(&u, s->master + i, 4);
+      if ((u & 0x7FFFFFFFu) > 0x7F800000u) {
+        s->bf[i] = static_cast<uint16_t>((u >> 16) | 0x40u);  // quiet NaN
+      } else {
+        s->bf[i] = static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+      }
+    }
+  });
+  return MT_OK;
+}
+
+void mt_host_store_destroy(mt_host_store* s) {
+  if (!s) return;
+  if (s->bf) cudaFreeHost(s->bf);
+  if (s->master) cudaFreeHost(s->master);
+  delete s;
+}
+
+}  // extern "C"
+
+// ======================================================================= engine
+namespace {
+
+using Clock = std::chrono::steady_clock;
+
+struct EventTimer : GemmTimer {
+  std::vector<cudaEvent_t> ev;
+  std::vector<double> flops;
+  size_t n = 0;
+  bool overflow = false;
+  void before(cudaStream_t st) override {
+    if (n + 2 > ev.size()) {
+      overflow = true;
+      return;
+    }
+    cudaEventRecord(ev[n], st);
+  }
+  void after(cudaStream_t st, double f) override {
+    if (overflow || n + 2 > ev.size()) return;
+    cudaEventRecord(ev[n + 1], st);
+    flops.push_back(f);
+    n += 2;
+  }
+};
+
+struct SinkItem {
+  int jb, layer, slab;
+};
+
+}  // namespace
+
+struct mt_engine {
+  Geom G;
+  mt_layer_cfg cfg;
+  int L, B, T, K, R, NS, NG, S;
+  int64_t M;
+  mt_engine_opts opts;
+  cudaStream_t cs, ps, os;
+  // device buffers
+  std::vector<mt_bf16*> slot;
+  std::vector<float*> dgrad;
+  std::vector<mt_bf16*> ckpt, seg;
+  mt_bf16 *act[2] = {nullptr, nullptr}, *gbuf[2] = {nullptr, nullptr}, *io[4] = {nullptr, nullptr, nullptr, nullptr};
+  void* lws = nullptr;
+  uint64_t lws_bytes = 0, dev_bytes = 0;
+  // host slab pool
+  std::vector<float*> slab;
+  std::mutex mu;
+  std::condition_variable cv;
+  std::vector<int> free_slabs;
+  std::deque<SinkItem> queue;
+  bool producer_done = false, abort = false, sink_finished = true;
+  mt_status sink_status = MT_OK;
+  std::thread sink_thread;
+  // schedule and events
+  std::vector<Use> uses;
+  std::vector<int> uslot, uload, prev_of_slot, load_of_use;
+  std::vector<cudaEvent_t> ready, done, g_ready, d2h_done;
+  cudaEvent_t fin = nullptr;
+  bool resident_loaded = false;
+  int64_t h2d_count = 0;
+  EventTimer timer;
+  mt_stats st;
+};
+
+namespace {
+
+mt_bf16* x_loc(mt_engine* e, int j, const mt_bf16* x0, mt_bf16* ytop) {
+  if (j == 0) return const_cast<mt_bf16*>(x0);
+  if (j == e->L) return ytop;
+  if (j % e->K == 0) return e->ckpt[j / e->K - 1];
+  return e->act[j % 2];
+}
+
+mt_status validate_opts(const mt_engine_opts* in, int L, mt_engine_opts* o) {
+  if (!in) return fail(MT_ERR_INVALID_ARG, "opts is NULL");
+  *o = *in;
+  if (o->ckpt_interval < 1) return fail(MT_ERR_INVALID_ARG, "ckpt_interval must be >= 1");
+  if (o->n_weight_slots < 0 || o->n_host_slabs < 0 || o->n_dev_grad_slabs < 0 || o->mlp_chunk < 0 ||
+      o->timeout_ms < 0 || o->fail_h2d_at < 0)
+    return fail(MT_ERR_INVALID_ARG, "engine options must be >= 0");
+  if (o->n_weight_slots == 0) o->n_weight_slots = std::max(2, o->ckpt_interval);
+  if (o->resident) o->n_weight_slots = L;
+  if (o->n_host_slabs == 0) o->n_host_slabs = 3;
+  if (o->n_dev_grad_slabs == 0) o->n_dev_grad_slabs = 2;
+  if (o->timeout_ms == 0) o->timeout_ms = 60000;
+  return MT_OK;
+}
+
+Bump carve_engine(const Geom& G, int L, int B, int T, const mt_engine_opts& o, void* base, uint64_t cap,
+                  mt_engine* e) {
+  const int64_t M = static_cast<int64_t>(B) * T;
+  const int K = o.ckpt_interval;
+  const int S = (L + K - 1) / K;
+  const int64_t rec = static_cast<int64_t>(G.off.record_elems);
+  Bump bp(base, cap);
+  for (int r = 0; r < o.n_weight_slots; ++r) {
+    mt_bf16* p = bp.take<mt_bf16>(rec);
+    if (e) e->slot.push_back(p);
+  }
+  for (int r = 0; r < o.n_dev_grad_slabs; ++r) {
+    float* p = bp.take<float>(rec);
+    if (e) e->dgrad.push_back(p);
+  }
+  for (int s = 1; s < S; ++s) {
+    mt_bf16* p = bp.take<mt_bf16>(M * G.H);
+    if (e) e->ckpt.push_back(p);
+  }
+  for (int s = 0; s < K - 1; ++s) {
+    mt_bf16* p = bp.take<mt_bf16>(M * G.H);
+    if (e) e->seg.push_back(p);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mt_bf16* a = bp.take<mt_bf16>(M * G.H);
+    mt_bf16* g = bp.take<mt_bf16>(M * G.H);
+    if (e) {
+      e->act[i] = a;
+      e->gbuf[i] = g;
+    }
+  }
+  for (int i = 0; i < 4; ++i) {
+    mt_bf16* p = bp.take<mt_bf16>(M * G.H);
+    if (e) e->io[i] = p;
+  }
+  return bp;
+}
+
+mt_status poll_event(cudaEvent_t ev, Clock::time_point deadline, const char* what) {
+  for (int spin = 0;; ++spin) {
+    cudaError_t r = cudaEventQuery(ev);
+    if (r == cudaSuccess) return MT_OK;
+    if (r != cudaErrorNotReady) return fail(MT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(r));
+    if (Clock::now() > deadline) return fail(MT_ERR_TIMEOUT, "%s: timed out", what);
+    if (spin > 64) std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+}
+
+mt_status poll_stream(cudaStream_t s, Clock::time_point deadline, const char* what) {
+  for (int spin = 0;; ++spin) {
+    cudaError_t r = cudaStreamQuery(s);
+    if (r == cudaSuccess) return MT_OK;
+    if (r != cudaErrorNotReady) return fail(MT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(r));
+    if (Clock::now() > deadline) return fail(MT_ERR_TIMEOUT, "%s: timed out", what);
+    if (spin > 64) std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+}
+
+void sink_loop(mt_engine* e, mt_grad_sink sink, void* user) {
+  const uint64_t rec = e->G.off.record_elems;
+  for (;;) {
+    SinkItem it;
+    {
+      std::unique_lock<std::mutex> lk(e->mu);
+      e->cv.wait(lk, [e] { return !e->queue.empty() || e->producer_done || e->abort; });
+      if (e->queue.empty() || e->abort) break;
+      it = e->queue.front();
+      e->queue.pop_front();
+    }
+    const auto deadline = Clock::now() + std::chrono::milliseconds(e->opts.timeout_ms);
+    mt_status s = poll_event(e->d2h_done[it.jb], deadline, "gradient offload");
+    if (s == MT_OK && sink) {
+      const auto t0 = Clock::now();
+      int32_t rc = sink(it.layer, e->slab[it.slab], rec, user);
+      e->st.sink_ms += std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
+      if (rc != 0) s = fail(MT_ERR_SINK, "gradient sink returned %d for layer %d", rc, it.layer);
+    }
+    std::lock_guard<std::mutex> lk(e->mu);
+    e->free_slabs.push_back(it.slab);
+    if (s != MT_OK) {
+      e->sink_status = s;
+      e->abort = true;
+    }
+    e->cv.notify_all();
+    if (s != MT_OK) break;
+  }
+  std::lock_guard<std::mutex> lk(e->mu);
+  e->sink_finished = true;
+  e->cv.notify_all();
+}
+
+// The schedule of one step, derived from the static use list.
+void prepare_schedule(mt_engine* e) {
+  e->uses = build_uses(e->L, e->K);
+  plan_slots(e->uses, e->R, e->uslot, e->uload);
+  const int n = static_cast<int>(e->uses.size());
+  e->prev_of_slot.assign(n, -1);
+  e->load_of_use.assign(n, -1);
+  std::vector<int> last_use(e->R, -1), last_load(e->R, -1);
+  for (int i = 0; i < n; ++i) {
+    const int s = e->uslot[i];
+    e->prev_of_slot[i] = last_use[s];
+    if (e->uload[i]) last_load[s] = i;
+    e->load_of_use[i] = last_load[s];
+    last_use[s] = i;
+  }
+}
+
+mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top, mt_bf16* y_top,
+                   mt_bf16* dx0, mt_grad_sink sink, void* user) {
+  const uint64_t rec = e->G.off.record_elems;
+  const int n = static_cast<int>(e->uses.size());
+  const bool skip_loads = e->opts.resident && e->resident_loaded;
+  int next_load = 0;
+  int jb = 0;  // backward index
+  mt_status status = MT_OK;
+  const auto timeout = std::chrono::milliseconds(e->opts.timeout_ms);
+
+  // sink thread for this step
+  {
+    std::lock_guard<std::mutex> lk(e->mu);
+    e->queue.clear();
+    e->producer_done = false;
+    e->abort = false;
+    e->sink_status = MT_OK;
+    e->sink_finished = false;
+    e->free_slabs.clear();
+    for (int i = 0; i < e->NS; ++i) e->free_slabs.push_back(i);
+  }
+  if (e->sink_thread.joinable()) e->sink_thread.join();  // finished: checked by the caller
+  e->sink_thread = std::thread(sink_loop, e, sink, user);
+
+  auto enqueue_loads = [&](int computed) -> mt_status {
+    // enqueue, in use order, every load whose slot's previous user has been enqueued
+    while (next_load < n) {
+      if (skip_loads || !e->uload[next_load]) {
+        ++next_load;
+        continue;
+      }
+      const int p = e->prev_of_slot[next_load];
+      if (p >= computed) break;
+      if (e->opts.fail_h2d_at > 0 && e->h2d_count + 1 == e->opts.fail_h2d_at) {
+        ++e->h2d_count;
+        return fail(MT_ERR_INJECTED, "injected failure of weight copy %lld", (long long)e->h2d_count);
+      }
+      if (p >= 0) MT_CUDA(cudaStreamWaitEvent(e->ps, e->done[p], 0));
+      const int layer = e->uses[next_load].layer;
+      MT_CUDA(cudaMemcpyAsync(e->slot[e->uslot[next_load]], mt_host_store_bf16(store, layer), rec * 2,
+                              cudaMemcpyHostToDevice, e->ps));
+      MT_CUDA(cudaEventRecord(e->ready[next_load], e->ps));
+      ++e->h2d_count;
+      e->st.h2d_bytes += rec * 2;
+      e->st.weight_loads += 1;
+      ++next_load;
+    }
+    return MT_OK;
+  };
+
+  for (int i = 0; i < n && status == MT_OK; ++i) {
+    {
+      std::lock_guard<std::mutex> lk(e->mu);
+      if (e->abort) {
+        status = e->sink_status != MT_OK ? e->sink_status : fail(MT_ERR_TIMEOUT, "step aborted");
+        break;
+      }
+    }
+    status = enqueue_loads(i);
+    if (status != MT_OK) break;
+    const Use u = e->uses[i];
+    const int l = u.layer;
+    const int s = l / e->K, a = s * e->K;
+    mt_bf16* w = e->slot[e->uslot[i]];
+    if (!skip_loads && e->load_of_use[i] >= 0) {
+      status = cuda_check(cudaStreamWaitEvent(e->cs, e->ready[e->load_of_use[i]], 0), "wait weights");
+      if (status != MT_OK) break;
+    }
+    if (u.kind == 0) {
+      status = mt_layer_fwd(&e->cfg, w, x_loc(e, l, x0, y_top), x_loc(e, l + 1, x0, y_top), e->B, e->T,
+                            e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs);
+      e->st.layer_fwd_calls++;
+    } else if (u.kind == 1) {
+      const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
+      status = mt_layer_fwd(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes,
+                            e->cs);
+      e->st.layer_fwd_calls++;
+    } else {
+      const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
+      const mt_bf16* dy = (jb == 0) ? dy_top : e->gbuf[(jb - 1) % 2];
+      mt_bf16* dx = (l == 0) ? dx0 : e->gbuf[jb % 2];
+      const int ns = jb % e->NG;
+      if (jb >= e->NG) {
+        status = cuda_check(cudaStreamWaitEvent(e->cs, e->d2h_done[jb - e->NG], 0), "wait staging slab");
+        if (status != MT_OK) break;
+      }
+      status = mt_layer_recompute_bwd(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
+                                      e->lws_bytes, e->cs);
+      e->st.layer_bwd_calls++;
+      if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
+      if (status == MT_OK) {
+        // take a pinned slab from the pool (bounded wait), then offload
+        int p = -1;
+        {
+          std::unique_lock<std::mutex> lk(e->mu);
+          const bool got = e->cv.wait_for(lk, timeout, [e] { return !e->free_slabs.empty() || e->abort; });
+          if (e->abort) {
+            status = e->sink_status != MT_OK ? e->sink_status : fail(MT_ERR_TIMEOUT, "step aborted");
+          } else if (!got) {
+            status = fail(MT_ERR_TIMEOUT, "no free gradient slab within %d ms", e->opts.timeout_ms);
+          } else {
+            p = e->free_slabs.back();
+            e->free_slabs.pop_back();
+          }
+        }
+        if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->g_ready[jb], 0), "wait g_ready");
+        if (status == MT_OK)
+          status = cuda_check(
+              cudaMemcpyAsync(e->slab[p], e->dgrad[ns], rec * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
+        if (status == MT_OK) status = cuda_check(cudaEventRecord(e->d2h_done[jb], e->os), "record d2h_done");
+        if (status == MT_OK) {
+          e->st.d2h_bytes += rec * 4;
+          std::lock_guard<std::mutex> lk(e->mu);
+          e->queue.push_back({jb, l, p});
+          e->cv.notify_all();
+        } else if (p >= 0) {
+          std::lock_guard<std::mutex> lk(e->mu);
+          e->free_slabs.push_back(p);
+        }
+      }
+      ++jb;
+    }
+    if (status != MT_OK) break;
+    status = cuda_check(cudaEventRecord(e->done[i], e->cs), "record done");
+  }
+  if (status == MT_OK) status = enqueue_loads(n);
+
+  // let the sink thread drain (bounded), then wait for the compute stream
+  {
+    std::unique_lock<std::mutex> lk(e->mu);
+    e->producer_done = true;
+    if (status != MT_OK) e->abort = true;
+    e->cv.notify_all();
+    const bool fin = e->cv.wait_for(lk, timeout * 2, [e] { return e->sink_finished; });
+    if (!fin && status == MT_OK) status = fail(MT_ERR_TIMEOUT, "gradient sink did not finish within the timeout");
+    if (status == MT_OK && e->sink_status != MT_OK) status = e->sink_status;
+  }
+  if (e->sink_finished && e->sink_thread.joinable()) e->sink_thread.join();
+  if (status == MT_OK) {
+    status = cuda_check(cudaEventRecord(e->fin, e->cs), "record fin");
+    if (status == MT_OK) status = poll_event(e->fin, Clock::now() + timeout, "compute stream");
+  }
+  if (status == MT_OK && e->opts.resident) e->resident_loaded = true;
+  return status;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t mt_engine_workspace_bytes(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B, int32_t T,
+                                   const mt_engine_opts* opts) {
+  Geom G;
+  mt_engine_opts o;
+  if (make_geom(cfg, &G) != MT_OK || n_layers <= 0 || validate_opts(opts, n_layers, &o) != MT_OK) return 0;
+  Bump bp = carve_engine(G, n_layers, B, T, o, nullptr, 0, nullptr);
+  const uint64_t lw = mt_layer_workspace_bytes(cfg, B, T, o.mlp_chunk);
+  if (lw == 0) return 0;
+  return bp.used + static_cast<uint64_t>(align_up(static_cast<int64_t>(lw), 256));
+}
+
+mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B, int32_t T,
+                           const mt_engine_opts* opts, void* dev_ws, uint64_t dev_ws_bytes, void* compute_stream,
+                           void* prefetch_stream, void* offload_stream, mt_engine** out) {
+  if (!out) return fail(MT_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  Geom G;
+  MT_TRY(make_geom(cfg, &G));
+  if (n_layers <= 0 || B <= 0 || T <= 0) return fail(MT_ERR_INVALID_ARG, "n_layers, B, T must be positive");
+  mt_engine_opts o;
+  MT_TRY(validate_opts(opts, n_layers, &o));
+  if (!compute_stream || !prefetch_stream || !offload_stream || compute_stream == prefetch_stream ||
+      compute_stream == offload_stream || prefetch_stream == offload_stream)
+    return fail(MT_ERR_INVALID_ARG, "compute, prefetch and offload must be three distinct non-default streams");
+  const uint64_t need = mt_engine_workspace_bytes(cfg, n_layers, B, T, &o);
+  if (need == 0) return fail(MT_ERR_INVALID_ARG, "layer workspace unavailable: %s", mt_last_error());
+  if (!dev_ws || !aligned16(dev_ws)) return fail(MT_ERR_ALIGNMENT, "device workspace must be 16-byte aligned");
+  if (dev_ws_bytes < need)
+    return fail(MT_ERR_WORKSPACE, "engine workspace %llu < %llu bytes", (unsigned long long)dev_ws_bytes,
+                (unsigned long long)need);
+  auto* e = new mt_engine();
+  e->G = G;
+  e->cfg = *cfg;
+  e->L = n_layers;
+  e->B = B;
+  e->T = T;
+  e->M = static_cast<int64_t>(B) * T;
+  e->opts = o;
+  e->K = o.ckpt_interval;
+  e->R = o.n_weight_slots;
+  e->NS = o.n_host_slabs;
+  e->NG = o.n_dev_grad_slabs;
+  e->S = (n_layers + e->K - 1) / e->K;
+  e->cs = as_stream(compute_stream);
+  e->ps = as_stream(prefetch_stream);
+  e->os = as_stream(offload_stream);
+  Bump bp = carve_engine(G, n_layers, B, T, o, dev_ws, dev_ws_bytes, e);
+  e->lws = static_cast<char*>(dev_ws) + bp.used;
+  e->lws_bytes = dev_ws_bytes - bp.used;
+  e->dev_bytes = need;
+  prepare_schedule(e);
+  auto cleanup = [e](mt_status s) {
+    mt_engine_destroy(e);
+    return s;
+  };
+  const uint64_t rec = G.off.record_elems;
+  for (int i = 0; i < e->NS; ++i) {
+    float* p = nullptr;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&p), rec * 4, cudaHostAllocPortable) != cudaSuccess) {
+      cudaGetLastError();
+      return cleanup(fail(MT_ERR_OOM, "pinned gradient slab allocation failed"));
+    }
+    e->slab.push_back(p);
+  }
+  const int n = static_cast<int>(e->uses.size());
+  auto mk = [](std::vector<cudaEvent_t>& v, int count) -> mt_status {
+    v.assign(count, nullptr);
+    for (int i = 0; i < count; ++i) MT_CUDA(cudaEventCreateWithFlags(&v[i], cudaEventDisableTiming));
+    return MT_OK;
+  };
+  mt_status s = mk(e->ready, n);
+  if (s == MT_OK) s = mk(e->done, n);
+  if (s == MT_OK) s = mk(e->g_ready, n_layers);
+  if (s == MT_OK) s = mk(e->d2h_done, n_layers);
+  if (s == MT_OK) s = cuda_check(cudaEventCreateWithFlags(&e->fin, cudaEventDisableTiming), "event");
+  if (s == MT_OK && o.time_gemms) {
+    e->timer.ev.assign(8192, nullptr);
+    for (auto& ev : e->timer.ev) {
+      s = cuda_check(cudaEventCreate(&ev), "timing event");
+      if (s != MT_OK) break;
+    }
+  }
+  if (s != MT_OK) return cleanup(s);
+  std::memset(&e->st, 0, sizeof(e->st));
+  e->st.device_bytes = need;
+  *out = e;
+  return MT_OK;
+}
+
+mt_status mt_stream_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top, mt_bf16* y_top,
+                         mt_bf16* dx0, mt_grad_sink sink, void* user) {
+  if (!e || !store || !x0 || !dy_top || !y_top || !dx0) return fail(MT_ERR_INVALID_ARG, "stream_step: NULL argument");
+  if (store->L != e->L || store->G.off.record_elems != e->G.off.record_elems)
+    return fail(MT_ERR_INVALID_ARG, "host store does not match the engine's layer count or shape");
+  if (!aligned16(x0) || !aligned16(dy_top) || !aligned16(y_top) || !aligned16(dx0))
+    return fail(MT_ERR_ALIGNMENT, "stream_step: activation pointers must be 16-byte aligned");
+  if (!e->sink_finished) return fail(MT_ERR_INVALID_ARG, "engine has an unfinished step; call mt_engine_reset");
+  const auto t0 = Clock::now();
+  const double f0 = exec_flops_counter();
+  const uint64_t k0 = launch_counter();
+  const uint64_t h2d0 = e->st.h2d_bytes, d2h0 = e->st.d2h_bytes;
+  e->st.sink_ms = 0;
+  e->timer.n = 0;
+  e->timer.flops.clear();
+  e->timer.overflow = false;
+  if (e->opts.time_gemms) set_gemm_timer(&e->timer);
+  mt_status s = run_step(e, store, x0, dy_top, y_top, dx0, sink, user);
+  set_gemm_timer(nullptr);
+  e->st.step_ms = std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
+  e->st.exec_flops = exec_flops_counter() - f0;
+  e->st.kernel_launches = launch_counter() - k0;
+  e->st.h2d_bytes -= h2d0;
+  e->st.d2h_bytes -= d2h0;
+  e->st.gemm_ms = 0;
+  e->st.gemm_flops = 0;
+  e->st.gemm_launches = 0;
+  if (s == MT_OK && e->opts.time_gemms) {
+    for (size_t k = 0; 2 * k + 1 < e->timer.n; ++k) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, e->timer.ev[2 * k], e->timer.ev[2 * k + 1]) == cudaSuccess) {
+        e->st.gemm_ms += ms;
+        e->st.gemm_flops += e->timer.flops[k];
+        e->st.gemm_launches += 1;
+      }
+    }
+  }
+  return s;
+}
+
+mt_status mt_stream_step_host(mt_engine* e, mt_host_store* store, const mt_bf16* x0_host, const mt_bf16* dy_top_host,
+                              mt_bf16* y_top_host, mt_bf16* dx0_host, mt_grad_sink sink, void* user) {
+  if (!e || !x0_host || !dy_top_host || !y_top_host || !dx0_host)
+    return fail(MT_ERR_INVALID_ARG, "stream_step_host: NULL argument");
+  const uint64_t bytes = static_cast<uint64_t>(e->M) * e->G.H * 2;
+  MT_CUDA(cudaMemcpyAsync(e->io[0], x0_host, bytes, cudaMemcpyHostToDevice, e->cs));
+  MT_CUDA(cudaMemcpyAsync(e->io[1], dy_top_host, bytes, cudaMemcpyHostToDevice, e->cs));
+  MT_TRY(mt_stream_step(e, store, e->io[0], e->io[1], e->io[2], e->io[3], sink, user));
+  MT_CUDA(cudaMemcpyAsync(y_top_host, e->io[2], bytes, cudaMemcpyDeviceToHost, e->cs));
+  MT_CUDA(cudaMemcpyAsync(dx0_host, e->io[3], bytes, cudaMemcpyDeviceToHost, e->cs));
+  MT_CUDA(cudaEventRecord(e->fin, e->cs));
+  MT_TRY(poll_event(e->fin, Clock::now() + std::chrono::milliseconds(e->opts.timeout_ms), "output copies"));
+  e->st.h2d_bytes += 2 * bytes;
+  e->st.d2h_bytes += 2 * bytes;
+  return MT_OK;
+}
+
+mt_status mt_engine_stats(const mt_engine* e, mt_stats* out) {
+  if (!e || !out) return fail(MT_ERR_INVALID_ARG, "NULL argument");
+  *out = e->st;
+  return MT_OK;
+}
+
+mt_status mt_engine_reset(mt_engine* e) {
+  if (!e) return fail(MT_ERR_INVALID_ARG, "engine is NULL");
+  const auto deadline = Clock::now() + std::chrono::milliseconds(e->opts.timeout_ms);
+  {
+    std::unique_lock<std::mutex> lk(e->mu);
+    e->abort = true;
+    e->producer_done = true;
+    e->cv.notify_all();
+    if (!e->cv.wait_until(lk, deadline, [e] { return e->sink_finished; }))
+      return fail(MT_ERR_TIMEOUT, "gradient sink still running");
+  }
+  if (e->sink_thread.joinable()) e->sink_thread.join();
+  MT_TRY(poll_stream(e->cs, deadline, "compute stream"));
+  MT_TRY(poll_stream(e->ps, deadline, "prefetch stream"));
+  MT_TRY(poll_stream(e->os, deadline, "offload stream"));
+  std::lock_guard<std::mutex> lk(e->mu);
+  e->abort = false;
+  e->queue.clear();
+  e->sink_status = MT_OK;
+  return MT_OK;
+}
+
+void mt_engine_destroy(mt_engine* e) {
+  if (!e) return;
+  {
+    std::unique_lock<std::mutex> lk(e->mu);
+    e->abort = true;
+    e->producer_done = true;
+    e->cv.notify_all();
+  }
+  if (e->sink_thread.joinable()) e->sink_thread.join();
+  cudaStreamSynchronize(e->cs);
+  cudaStreamSynchronize(e->ps);
+  cudaStreamSynchronize(e->os);
+  for (auto* v : {&e->ready, &e->done, &e->g_ready, &e->d2h_done, &e->timer.ev})
+    for (auto ev : *v)
+      if (ev) cudaEventDestroy(ev);
+  if (e->fin) cudaEventDestroy(e->fin);
+  for (float* p : e->slab) cudaFreeHost(p);
+  delete e;
+}
+
+}  // extern "C"

@@ -1,0 +1,533 @@
+// C = A * B^T on the sm_100a tensor cores: TMA-fed, tcgen05.mma with the
+// accumulator in tensor memory, persistent and warp-specialised.
+//
+// This is the dense contraction of every projection of the decoder layer
+// (QKV, O, gate/up, down) in its three uses: the forward Y = X W^T (both
+// operands K-major), the input gradient dX = dY W (B is MN-major) and the
+// weight gradient dW = dY^T X (both MN-major), which the layer template of
+// the MegaTrain pages ("stateless layer templates", abstract) runs for every
+// streamed layer.
+//
+// Design
+// - Tile 128 x 256 x 64 (bf16), 4-stage shared-memory ring, one CTA per SM,
+//   persistent over output tiles (grouped raster, 16 row-blocks per group).
+// - Warp 0: TMA producer. Warp 1: TMEM allocation and the MMA issuer.
+//   Warps 2-5: epilogue (tcgen05.ld of the fp32 accumulator, bias/residual,
+//   bf16 or fp32 store).
+// - Two 256-column accumulators in TMEM (512 columns): the epilogue of one
+//   tile overlaps the main loop of the next.
+// - Operands are staged with 128-byte swizzle. K-major tiles are one TMA box
+//   of 64 (K) x rows; MN-major tiles are boxes of 64 (M or N) x 64 (K) placed
+//   8 KiB apart, which is the descriptor's leading-byte offset.
+// - Every mbarrier wait is bounded (4 s); when one runs out the kernel sets
+//   the device error word and all roles leave their loops, free TMEM and exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "mt_internal.h"
+
+namespace mt {
+GemmTimer* current_gemm_timer();
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_TILE = BM * BK * 2;  // 16 KiB
+constexpr int B_TILE = BN * BK * 2;  // 32 KiB
+constexpr int MN_BOX = 64 * BK * 2;  // one 64 x 64 MN-major box: 8 KiB
+constexpr int SMEM_TILES = STAGES * (A_TILE + B_TILE);
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;
+constexpr unsigned long long WAIT_NS = 4000000000ull;
+
+struct EpiArgs {
+  void* C;
+  const __nv_bfloat16* bias;
+  const __nv_bfloat16* res;
+  int64_t ldc, ldr;
+  int M, N, K;
+  int c_f32, accumulate;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on the phase with the given parity. Returns false when it ran
+// out (or another role already aborted); the first timeout records `code`.
+__device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* err, int code) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 127u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > WAIT_NS) {
+        *abort_flag = 1;
+        atomicCAS(err, 0, code);
+        return false;
+      }
+    }
+  }
+}
+
+// Lane 0 waits, the whole warp gets the outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* err,
+                                          int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, err, code) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (sm_100 layout: start>>4 in [0,14),
+// leading-byte offset>>4 in [16,30), stride-byte offset>>4 in [32,46),
+// version 1 at bit 46, swizzle mode in [61,64) with 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and
+// B bf16 (bits 7-9 and 10-12 = 1), A/B major bits 15/16, N>>3 at 17, M>>4 at 24.
+__host__ __device__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+  constexpr int G = 16;
+  const int group_tiles = G * num_n;
+  const int g = t / group_tiles;
+  const int first_m = g * G;
+  const int gm = min(num_m - first_m, G);
+  const int r = t - g * group_tiles;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Epilogue of one 32-column chunk of one output row.
+__device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  const bool full = col0 + 32 <= ep.N;
+  if (full) {
+    if (ep.bias) {
+      const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = __ldg(bp + q);
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[q * 8 + j] += bf2f(h[j]);
+      }
+    }
+    if (ep.res) {
+      const uint4* rp = reinterpret_cast<const uint4*>(ep.res + static_cast<int64_t>(row) * ep.ldr + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = rp[q];
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[q * 8 + j] += bf2f(h[j]);
+      }
+    }
+    if (ep.c_f32) {
+      float4* cp = reinterpret_cast<float4*>(static_cast<float*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 o = make_float4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+        if (ep.accumulate) {
+          float4 p = cp[q];
+          o.x += p.x;
+          o.y += p.y;
+          o.z += p.z;
+          o.w += p.w;
+        }
+        cp[q] = o;
+      }
+    } else {
+      uint4* cp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc +
+                                           col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(v[q * 8 + 2 * j], v[q * 8 + 2 * j + 1]);
+        cp[q] = u;
+      }
+    }
+  } else {
+    for (int j = 0; j < 32; ++j) {
+      const int col = col0 + j;
+      if (col >= ep.N) break;
+      float x = v[j];
+      if (ep.bias) x += bf2f(ep.bias[col]);
+      if (ep.res) x += bf2f(ep.res[static_cast<int64_t>(row) * ep.ldr + col]);
+      if (ep.c_f32) {
+        float* cp = static_cast<float*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col;
+        *cp = ep.accumulate ? *cp + x : x;
+      } else {
+        static_cast<__nv_bfloat16*>(ep.C)[static_cast<int64_t>(row) * ep.ldc + col] = __float2bfloat16_rn(x);
+      }
+    }
+  }
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, EpiArgs ep,
+                int32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
+  uint64_t* full = bars;                // TMA -> MMA, one per stage
+  uint64_t* empty = bars + STAGES;      // MMA -> TMA, one per stage
+  uint64_t* tfull = bars + 2 * STAGES;  // MMA -> epilogue, one per accumulator
+  uint64_t* tempty = tfull + 2;         // epilogue -> MMA, one per accumulator
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (ep.M + BM - 1) / BM, num_n = (ep.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (ep.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 128);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      const int m0 = mb * BM, n0 = nb * BN;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!warp_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&full[s]);
+          const uint32_t a_dst = smem_u32(sA + s * A_TILE), b_dst = smem_u32(sB + s * B_TILE);
+          const int k0 = kb * BK;
+          // Boxes that lie wholly past M or N are skipped: those rows of the
+          // tile only feed output rows/columns that are never stored.
+          uint32_t bytes = 0;
+          if (!A_MN) {
+            bytes += A_TILE;
+          } else {
+            for (int j = 0; j < BM / 64; ++j)
+              if (m0 + 64 * j < ep.M) bytes += MN_BOX;
+          }
+          if (!B_MN) {
+            bytes += B_TILE;
+          } else {
+            for (int j = 0; j < BN / 64; ++j)
+              if (n0 + 64 * j < ep.N) bytes += MN_BOX;
+          }
+          mbar_expect_tx(fb, bytes);
+          if (!A_MN) {
+            tma_load_2d(a_dst, &tmA, fb, k0, m0);
+          } else {
+            for (int j = 0; j < BM / 64; ++j)
+              if (m0 + 64 * j < ep.M) tma_load_2d(a_dst + j * MN_BOX, &tmA, fb, m0 + 64 * j, k0);
+          }
+          if (!B_MN) {
+            tma_load_2d(b_dst, &tmB, fb, k0, n0);
+          } else {
+            for (int j = 0; j < BN / 64; ++j)
+              if (n0 + 64 * j < ep.N) tma_load_2d(b_dst + j * MN_BOX, &tmB, fb, n0 + 64 * j, k0);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = make_idesc(A_MN, B_MN);
+    uint32_t it = 0;
+    int tl = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tl) {
+      const int ab = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1u;
+      if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
+      fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!warp_wait(smem_u32(&full[s]), ph, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        if (lane == 0) {
+          const uint32_t a_base = smem_u32(sA + s * A_TILE), b_base = smem_u32(sB + s * B_TILE);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // K-major: advance 16 elements (32 bytes) inside the swizzled row.
+            // MN-major: advance 16 K-rows (two 8-row groups of 1 KiB).
+            const uint64_t ad = A_MN ? smem_desc(a_base + kk * 2048, MN_BOX, 1024) : smem_desc(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(b_base + kk * 2048, MN_BOX, 1024) : smem_desc(b_base + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&empty[s]));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&tfull[ab]));
+      __syncwarp();
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are readable by this warp
+    int tl = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
+      const int ab = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1u;
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
+      fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        if (col0 >= ep.N) break;  // uniform across the warp
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN + c * 32), r);
+        if (row < ep.M) store_chunk(ep, row, col0, r);
+      }
+      fence_before();
+      mbar_arrive(smem_u32(&tempty[ab]));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+mt_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                   uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a %llu x %llu tensor, ld %llu", int(r),
+                (unsigned long long)inner, (unsigned long long)outer, (unsigned long long)ld_elems);
+  return MT_OK;
+}
+
+template <bool A_MN, bool B_MN>
+mt_status launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return fail(MT_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(attr_err));
+  const int num_tiles = ((ep.M + BM - 1) / BM) * ((ep.N + BN - 1) / BN);
+  const int grid = std::min(num_tiles, num_sms());
+  int32_t* err = device_error_word();
+  if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
+  gemm_kernel<A_MN, B_MN><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, ep, err);
+  return launch_check("gemm_kernel");
+}
+
+}  // namespace
+
+mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn, void* C,
+                      int64_t ldc, bool c_f32, bool accumulate, int64_t M, int64_t N, int64_t K,
+                      const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, cudaStream_t st) {
+  if (M == 0 || N == 0) return MT_OK;
+  CUtensorMap ta, tb;
+  if (!a_mn)
+    MT_TRY(make_map(&ta, A, K, M, lda, 64, BM));
+  else
+    MT_TRY(make_map(&ta, A, M, K, lda, 64, 64));
+  if (!b_mn)
+    MT_TRY(make_map(&tb, B, K, N, ldb, 64, BN));
+  else
+    MT_TRY(make_map(&tb, B, N, K, ldb, 64, 64));
+  EpiArgs ep;
+  ep.C = C;
+  ep.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  ep.res = reinterpret_cast<const __nv_bfloat16*>(residual);
+  ep.ldc = ldc;
+  ep.ldr = ldr;
+  ep.M = static_cast<int>(M);
+  ep.N = static_cast<int>(N);
+  ep.K = static_cast<int>(K);
+  ep.c_f32 = c_f32 ? 1 : 0;
+  ep.accumulate = accumulate ? 1 : 0;
+  const double flops = 2.0 * double(M) * double(N) * double(K);
+  GemmTimer* tm = current_gemm_timer();
+  if (tm) tm->before(st);
+  mt_status s;
+  if (!a_mn && !b_mn)
+    s = launch_t<false, false>(ta, tb, ep, st);
+  else if (!a_mn && b_mn)
+    s = launch_t<false, true>(ta, tb, ep, st);
+  else if (a_mn && !b_mn)
+    s = launch_t<true, false>(ta, tb, ep, st);
+  else
+    s = launch_t<true, true>(ta, tb, ep, st);
+  if (tm) tm->after(st, flops);
+  add_exec_flops(flops);
+  return s;
+}
+
+}  // namespace mt
+
+using namespace mt;
+
+extern "C" mt_status mt_gemm_bf16(const mt_bf16* A, int64_t lda, int32_t a_mn_major, const mt_bf16* Bm, int64_t ldb,
+                                  int32_t b_mn_major, void* C, int64_t ldc, int32_t c_f32, int32_t accumulate,
+                                  int64_t M, int64_t N, int64_t K, const mt_bf16* bias, const mt_bf16* residual,
+                                  int64_t ldr, void* stream) {
+  if (!A || !Bm || !C) return fail(MT_ERR_INVALID_ARG, "A, B and C must not be NULL");
+  if (M < 0 || N < 0 || K <= 0) return fail(MT_ERR_INVALID_ARG, "need M, N >= 0 and K > 0");
+  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return fail(MT_ERR_INVALID_ARG, "dimension too large");
+  if (accumulate && !c_f32) return fail(MT_ERR_INVALID_ARG, "accumulate needs an fp32 C");
+  const int64_t a_inner = a_mn_major ? M : K, b_inner = b_mn_major ? N : K;
+  if (lda < a_inner || ldb < b_inner || ldc < N || (residual && ldr < N))
+    return fail(MT_ERR_INVALID_ARG, "leading dimension smaller than the row it holds");
+  if (!aligned16(A) || !aligned16(Bm) || !aligned16(C) || (bias && !aligned16(bias)) ||
+      (residual && !aligned16(residual)))
+    return fail(MT_ERR_ALIGNMENT, "gemm pointers must be 16-byte aligned");
+  if (lda % 8 || ldb % 8 || ldc % 8 || (residual && ldr % 8))
+    return fail(MT_ERR_ALIGNMENT, "leading dimensions must be multiples of 8 elements");
+  return gemm_launch(A, lda, a_mn_major != 0, Bm, ldb, b_mn_major != 0, C, ldc, c_f32 != 0, accumulate != 0, M, N, K,
+                     bias, residual, ldr, as_stream(stream));
+}

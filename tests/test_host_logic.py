@@ -1,0 +1,138 @@
+"""Host-side logic that needs no GPU: the C-ABI library loads and exports every
+entry point of include/mt.h, the layer record geometry, the streaming
+schedule, argument validation, and the throughput formula."""
+import json
+import os
+import re
+
+import pytest
+
+from host_offloaded_layer_b200 import _lib as L
+from host_offloaded_layer_b200 import metrics
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+QWEN7B = dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944)
+QWEN14B = dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824)
+TINY = dict(hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=688)
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "mt.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(mt_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(n for n in names if n != "mt_grad_sink"))
+
+
+def test_library_exports_every_declared_entry_point(lib):
+    names = _declared_functions()
+    assert len(names) >= 30
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in L._SIGS, f"binding lacks {n}"
+
+
+def test_param_count_reproduces_table5_depth_study():
+    g = json.load(open(os.path.join(GOLDEN, "table5_depth.json")))
+    cfg = L.make_cfg(g["hidden"], g["n_q_heads"], g["n_kv_heads"], g["head_dim"], g["ffn"])
+    p_layer = L.mt_layer_param_count(cfg)
+    assert p_layer == 233057792
+    rows = g["rows"]
+    # per-layer count from the depth deltas alone (no vocabulary assumption)
+    for (l0, p0), (l1, p1) in zip(rows, rows[1:]):
+        assert abs((p1 - p0) * 1e9 / (l1 - l0) - p_layer) / p_layer < 5e-3
+    # totals with the untied embedding + head of the Qwen2.5 vocabulary
+    for layers, billions in rows:
+        total = layers * p_layer + 2 * 152064 * g["hidden"]
+        assert abs(total / 1e9 - billions) <= 0.01
+
+
+def test_record_layout_contiguity_and_alignment():
+    for shape in (QWEN7B, QWEN14B, TINY):
+        cfg = L.make_cfg(**shape)
+        o = L.mt_layer_param_offsets(cfg)
+        H, F = shape["hidden"], shape["ffn"]
+        hq = shape["n_q_heads"] * shape["head_dim"]
+        hkv = shape["n_kv_heads"] * shape["head_dim"]
+        assert o.wk == o.wq + hq * H and o.wv == o.wk + hkv * H
+        assert o.bk == o.bq + hq and o.bv == o.bk + hkv
+        assert o.wu == o.wg + F * H
+        for blk in (o.g1, o.wq, o.bq, o.wo, o.g2, o.wg, o.wd, o.record_elems):
+            assert blk % 128 == 0
+        ends = [o.g1 + H, o.wv + hkv * H, o.bv + hkv, o.wo + H * hq, o.g2 + H, o.wu + F * H, o.wd + H * F]
+        starts = [o.g1, o.wq, o.bq, o.wo, o.g2, o.wg, o.wd]
+        for a, b in zip(ends[:-1], starts[1:]):
+            assert a <= b
+        assert ends[-1] <= o.record_elems
+        assert o.param_count == L.mt_layer_param_count(cfg)
+    assert L.mt_layer_param_count(L.make_cfg(**QWEN14B)) == 275268608
+    assert L.mt_layer_param_count(L.make_cfg(**TINY)) == 726016
+
+
+def test_device_workspace_does_not_grow_with_depth():
+    """MegaTrain Table 5: device allocation is the same at every depth."""
+    cfg = L.make_cfg(**QWEN7B)
+    opts = L.make_opts(ckpt_interval=4)
+    base = L.mt_engine_workspace_bytes(cfg, 4, 1, 1024, opts)
+    assert base > 0
+    # only the checkpoint stash (one activation per K layers) depends on depth
+    act = 1 * 1024 * 3584 * 2
+    for layers in (28, 42, 180):
+        extra = L.mt_engine_workspace_bytes(cfg, layers, 1, 1024, opts) - base
+        assert extra == ((layers + 3) // 4 - 1) * act
+
+
+@pytest.mark.parametrize("n_layers,K,R", [(4, 4, 4), (28, 4, 4), (6, 2, 2), (5, 1, 2), (7, 3, 3), (3, 4, 1)])
+def test_schedule_holds_each_layer_when_used(n_layers, K, R):
+    layer, kind, slot, load = L.mt_schedule(n_layers, K, R)
+    # forward 0..L-1, then per segment: re-forward of all but the last, backward descending
+    assert layer[:n_layers] == list(range(n_layers)) and set(kind[:n_layers]) == {0}
+    bwd = [l for l, k in zip(layer, kind) if k == 2]
+    assert bwd == list(range(n_layers - 1, -1, -1))
+    holds = [None] * R
+    loads = 0
+    for i in range(len(layer)):
+        assert 0 <= slot[i] < R
+        if load[i]:
+            holds[slot[i]] = layer[i]
+            loads += 1
+        assert holds[slot[i]] == layer[i]
+        if i > 0 and R > 1:
+            assert not (load[i] and slot[i] == slot[i - 1]), "a load must not evict the layer in use"
+    # with a K-slot ring each layer streams in at most twice per step (forward and
+    # its backward segment); a single buffer may also reload for the re-forward
+    assert loads <= (2 if R >= K else 3) * n_layers
+    if R >= n_layers:
+        assert loads == n_layers
+
+
+def test_invalid_arguments_are_rejected_without_a_gpu():
+    with pytest.raises(L.MTError) as e:
+        L.mt_layer_param_offsets(L.make_cfg(256, 4, 3, 64, 688))
+    assert e.value.name == "MT_ERR_INVALID_ARG"
+    assert L.mt_layer_param_count(L.make_cfg(0, 4, 2, 64, 688)) == 0
+    with pytest.raises(L.MTError) as e:
+        L.mt_gemm_bf16(None, 8, 0, None, 8, 0, None, 8, 0, 0, 8, 8, 8)
+    assert e.value.name == "MT_ERR_INVALID_ARG"
+    with pytest.raises(L.MTError) as e:
+        L.mt_gemm_bf16(16, 8, 0, 16, 8, 0, 16, 8, 0, 1, 8, 8, 8)  # accumulate into bf16
+    assert e.value.name == "MT_ERR_INVALID_ARG"
+    with pytest.raises(L.MTError) as e:
+        L.mt_gemm_bf16(16, 12, 0, 16, 8, 0, 16, 8, 0, 0, 8, 8, 8)  # lda not a multiple of 8
+    assert e.value.name == "MT_ERR_ALIGNMENT"
+    assert L.mt_layer_workspace_bytes(L.make_cfg(256, 4, 2, 64, 688), 0, 128, 0) == 0
+    with pytest.raises(L.MTError) as e:
+        L.mt_attention_fwd(16, 512, 16, 256, 16, 1, 8, 4, 2, 96)
+    assert e.value.name == "MT_ERR_UNSUPPORTED"
+    opts = L.make_opts(ckpt_interval=0)
+    assert L.mt_engine_workspace_bytes(L.make_cfg(**TINY), 2, 1, 8, opts) == 0
+
+
+def test_tflops_formula_reproduces_table7_long_context_rows():
+    g = json.load(open(os.path.join(GOLDEN, "table7_longctx.json")))
+    m = g["model"]
+    for r in g["rows"]:
+        tf = metrics.sustained_tflops(m["N"], m["L"], m["H"], r["B"], r["T"], r["step_s"])
+        assert abs(tf - r["tflops"]) / r["tflops"] < 1e-3, (r, tf)
+    assert metrics.tokens_per_s(96, 1024, 2.0) == 49152.0

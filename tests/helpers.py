@@ -9,6 +9,19 @@ from host_offloaded_layer_b200 import synth
 TOL = 2e-2  # relative Frobenius error per tensor (bf16 operands, fp32 accumulation)
 
 
+def branch_tol(x, y_ref) -> float:
+    """Error budget of a residual branch (Y - X) when the residual stream is stored in bf16.
+
+    The GPU stores the layer's two residual sums (x2 and y) as bf16. The error of
+    rounding the oracle's own Y to bf16, e_r = ||bf16(Y) - Y||, measures one such
+    rounding; two of them, with a factor 2 of slack each, are allowed on top of
+    the parity tolerance, relative to the branch ||Y - X||."""
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y_ref, dtype=np.float64)
+    e_r = np.linalg.norm(synth.bf16_round(y.astype(np.float32)).astype(np.float64) - y)
+    return TOL + 4.0 * e_r / max(np.linalg.norm(y - x), 1e-30)
+
+
 def rel(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)

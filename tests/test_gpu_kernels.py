@@ -40,7 +40,7 @@ def test_gemm_layouts_match_fp64_matmul(a_mn, b_mn, M, N, K):
     Bm = B64.T if b_mn else B64   # logical [N, K]
     ref = Am @ Bm.T
     dA, dB = H.dev_bf16(A), H.dev_bf16(B)
-    ldc = N + 8
+    ldc = (N + 7) // 8 * 8 + 8
     C = torch.zeros(M, ldc, dtype=torch.float32, device="cuda")
     L.mt_gemm_bf16(dA, lda, a_mn, dB, ldb, b_mn, C, ldc, 1, 0, M, N, K)
     torch.cuda.synchronize()

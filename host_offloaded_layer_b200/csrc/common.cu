@@ -111,7 +111,9 @@ mt_status make_geom(const mt_layer_cfg* cfg, Geom* g) {
 // ------------------------------------------------------------- schedule
 // Uses in compute order: forward 0..L-1; then for each segment s from last to
 // first (layers [sK, min(sK+K, L))): re-forward of all but its last layer,
-// then recompute+backward from its last layer down to its first.
+// then recompute+backward from its last layer down to its first. The last
+// segment needs no re-forward: the forward writes its inner activations
+// straight into the segment buffers, which the backward reads.
 struct Use {
   int32_t layer, kind;
 };
@@ -122,7 +124,8 @@ std::vector<Use> build_uses(int L, int K) {
   int S = (L + K - 1) / K;
   for (int s = S - 1; s >= 0; --s) {
     int a = s * K, b = std::min(L, a + K);
-    for (int l = a; l < b - 1; ++l) u.push_back({l, 1});
+    if (s != S - 1)
+      for (int l = a; l < b - 1; ++l) u.push_back({l, 1});
     for (int l = b - 1; l >= a; --l) u.push_back({l, 2});
   }
   return u;

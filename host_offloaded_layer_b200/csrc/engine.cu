@@ -37,6 +37,9 @@ struct Use {
 };
 std::vector<Use> build_uses(int L, int K);
 void plan_slots(const std::vector<Use>& u, int R, std::vector<int>& slot, std::vector<int>& load);
+mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
+                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done);
 }  // namespace mt
 
 using namespace mt;
@@ -197,7 +200,7 @@ struct mt_engine {
   // schedule and events
   std::vector<Use> uses;
   std::vector<int> uslot, uload, prev_of_slot, load_of_use;
-  std::vector<cudaEvent_t> ready, done, g_ready, d2h_done;
+  std::vector<cudaEvent_t> ready, done, g_ready, d2h_done, mlp_done;
   cudaEvent_t fin = nullptr;
   bool resident_loaded = false;
   int64_t h2d_count = 0;
@@ -406,8 +409,11 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       if (status != MT_OK) break;
     }
     if (u.kind == 0) {
-      status = mt_layer_fwd(&e->cfg, w, x_loc(e, l, x0, y_top), x_loc(e, l + 1, x0, y_top), e->B, e->T,
-                            e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs);
+      // inside the last segment the forward keeps its activations in the segment buffers
+      const int a_last = (e->S - 1) * e->K;
+      const mt_bf16* xin = (l > a_last) ? e->seg[l - a_last - 1] : x_loc(e, l, x0, y_top);
+      mt_bf16* xout = (l + 1 < e->L && l + 1 > a_last) ? e->seg[l - a_last] : x_loc(e, l + 1, x0, y_top);
+      status = mt_layer_fwd(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs);
       e->st.layer_fwd_calls++;
     } else if (u.kind == 1) {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
@@ -423,8 +429,8 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         status = cuda_check(cudaStreamWaitEvent(e->cs, e->d2h_done[jb - e->NG], 0), "wait staging slab");
         if (status != MT_OK) break;
       }
-      status = mt_layer_recompute_bwd(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
-                                      e->lws_bytes, e->cs);
+      status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
+                                      e->lws_bytes, e->cs, e->mlp_done[jb]);
       e->st.layer_bwd_calls++;
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
       if (status == MT_OK) {
@@ -442,10 +448,18 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
             e->free_slabs.pop_back();
           }
         }
+        // two pieces: the MLP weights' gradients (the record's tail from Wg on) as soon as
+        // the MLP backward is done, then the rest when the layer is done
+        const uint64_t split = e->G.off.wg;
+        if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->mlp_done[jb], 0), "wait mlp_done");
+        if (status == MT_OK)
+          status = cuda_check(cudaMemcpyAsync(e->slab[p] + split, e->dgrad[ns] + split, (rec - split) * 4,
+                                              cudaMemcpyDeviceToHost, e->os),
+                              "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->g_ready[jb], 0), "wait g_ready");
         if (status == MT_OK)
           status = cuda_check(
-              cudaMemcpyAsync(e->slab[p], e->dgrad[ns], rec * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
+              cudaMemcpyAsync(e->slab[p], e->dgrad[ns], split * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaEventRecord(e->d2h_done[jb], e->os), "record d2h_done");
         if (status == MT_OK) {
           e->st.d2h_bytes += rec * 4;
@@ -561,6 +575,7 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
   if (s == MT_OK) s = mk(e->done, n);
   if (s == MT_OK) s = mk(e->g_ready, n_layers);
   if (s == MT_OK) s = mk(e->d2h_done, n_layers);
+  if (s == MT_OK) s = mk(e->mlp_done, n_layers);
   if (s == MT_OK) s = cuda_check(cudaEventCreateWithFlags(&e->fin, cudaEventDisableTiming), "event");
   if (s == MT_OK && o.time_gemms) {
     e->timer.ev.assign(8192, nullptr);
@@ -673,7 +688,7 @@ void mt_engine_destroy(mt_engine* e) {
   cudaStreamSynchronize(e->cs);
   cudaStreamSynchronize(e->ps);
   cudaStreamSynchronize(e->os);
-  for (auto* v : {&e->ready, &e->done, &e->g_ready, &e->d2h_done, &e->timer.ev})
+  for (auto* v : {&e->ready, &e->done, &e->g_ready, &e->d2h_done, &e->mlp_done, &e->timer.ev})
     for (auto ev : *v)
       if (ev) cudaEventDestroy(ev);
   if (e->fin) cudaEventDestroy(e->fin);

@@ -18,6 +18,9 @@
 
 namespace mt {
 
+mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
+                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done);
 mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, int64_t, int, float, cudaStream_t);
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
@@ -147,6 +150,17 @@ mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_b
 mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
                                  uint64_t ws_bytes, void* stream) {
+  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr);
+}
+
+}  // extern "C"
+
+// The layer backward; when mlp_done is given it is recorded on the stream as
+// soon as the MLP weights' gradients (Wg, Wu, Wd) are final.
+mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x,
+                                     const mt_bf16* dy, mt_bf16* dx, float* dw_dev, int32_t B, int32_t T,
+                                     int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream,
+                                     cudaEvent_t mlp_done) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
   if (!w_dev || !x || !dy || !dx || !dw_dev || !ws) return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: NULL pointer");
@@ -189,6 +203,7 @@ mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, 
     MT_TRY(gemm_launch(w.gu, 2 * G.F, false, w_dev + O.wg, G.H, true, w.dh2 + r0 * G.H, G.H, false, false, rows, G.H,
                        2 * G.F, nullptr, nullptr, 0, st));
   }
+  if (mlp_done) MT_CUDA(cudaEventRecord(mlp_done, st));
   // dx2 = dy + RMSNorm2^T(dh2); dg2
   MT_TRY(rmsnorm_bwd_launch(w.dh2, w.x2, w_dev + O.g2, w.rstd2, dy, w.dx2, dw_dev + O.g2, M, H, w.red, st));
   // dWo = dx2^T o ; do = dx2 Wo
@@ -210,5 +225,3 @@ mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, 
   MT_TRY(rmsnorm_bwd_launch(w.dh2, x, w_dev + O.g1, w.rstd1, w.dx2, dx, dw_dev + O.g1, M, H, w.red, st));
   return MT_OK;
 }
-
-}  // extern "C"

@@ -28,8 +28,8 @@ def _check_dev_error():
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 300, 136), (2048, 4096, 512), (96, 40, 1000)])
 def test_gemm_layouts_match_fp64_matmul(a_mn, b_mn, M, N, K):
     import torch
-    lda = (M if a_mn else K) + 8
-    ldb = (N if b_mn else K) + 16
+    lda = ((M if a_mn else K) + 7) // 8 * 8 + 8
+    ldb = ((N if b_mn else K) + 7) // 8 * 8 + 16
     a_rows, a_cols = (K, M) if a_mn else (M, K)
     b_rows, b_cols = (K, N) if b_mn else (N, K)
     A = _bits(1, 1, a_rows * lda).reshape(a_rows, lda)

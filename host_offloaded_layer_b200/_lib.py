@@ -72,6 +72,7 @@ _SIGS = {
     "mt_rmsnorm_fwd": (c_i32, [_P, _P, _P, _P, c_i64, c_i32, c_f32, _P]),
     "mt_rmsnorm_bwd_workspace_bytes": (c_u64, [c_i64, c_i32]),
     "mt_rmsnorm_bwd": (c_i32, [_P, _P, _P, _P, _P, _P, _P, c_i64, c_i32, _P, c_u64, _P]),
+    "mt_rmsnorm_bwd_noalloc": (c_i32, [_P, _P, _P, _P, _P, _P, _P, c_i64, c_i32, _P]),
     "mt_rope": (c_i32, [_P, c_i64, c_i32, c_i32, c_i32, c_i32, c_f32, c_i32, _P]),
     "mt_swiglu_fwd": (c_i32, [_P, _P, c_i64, c_i32, _P]),
     "mt_swiglu_bwd": (c_i32, [_P, _P, _P, c_i64, c_i32, _P]),
@@ -199,6 +200,11 @@ def mt_rmsnorm_bwd_workspace_bytes(rows, H) -> int:
 def mt_rmsnorm_bwd(dy, x, g, rstd, dres, dx, dg, rows, H, ws, ws_bytes, stream=None):
     _check(load().mt_rmsnorm_bwd(_ptr(dy), _ptr(x), _ptr(g), _ptr(rstd), _ptr(dres), _ptr(dx), _ptr(dg), rows, H,
                                  _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def mt_rmsnorm_bwd_noalloc(dy, x, g, rstd, dres, dx, dg, rows, H, stream=None):
+    _check(load().mt_rmsnorm_bwd_noalloc(_ptr(dy), _ptr(x), _ptr(g), _ptr(rstd), _ptr(dres), _ptr(dx), _ptr(dg), rows,
+                                         H, _stream(stream)))
 
 
 def mt_rope(x, ld, B, T, n_heads, head_dim, theta, inverse, stream=None):

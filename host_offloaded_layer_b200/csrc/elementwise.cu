@@ -3,6 +3,8 @@
 // (bias and norm-gain gradients). Each is a single pass over its operands in
 // HBM with 16-byte vector accesses; reductions over tokens use per-block
 // partial rows reduced in a fixed order, so results are bitwise repeatable.
+#include <mutex>
+
 #include "mt_internal.h"
 
 namespace mt {
@@ -371,3 +373,51 @@ mt_status mt_colsum(const mt_bf16* X, int64_t rows, int64_t cols, int64_t ld, fl
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// mt_rmsnorm_bwd_noalloc: the RMSNorm backward for callers that cannot give a
+// workspace. Its partial-sum scratch is this file's own device array.
+namespace {
+
+constexpr int64_t NOALLOC_SCRATCH_FLOATS = int64_t(1) << 21;  // 8 MiB per device
+static __device__ __align__(256) float g_rmsnorm_scratch[NOALLOC_SCRATCH_FLOATS];
+
+// Device address of g_rmsnorm_scratch, looked up once per device with that
+// device current (in host code the symbol is only a host-side stand-in).
+mt_status noalloc_scratch(float** out) {
+  static std::mutex mu;
+  static float* addr[64] = {nullptr};
+  int dev = 0;
+  MT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MT_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    MT_CUDA(cudaGetSymbolAddress(&p, g_rmsnorm_scratch));
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return MT_OK;
+}
+
+}  // namespace
+
+extern "C" mt_status mt_rmsnorm_bwd_noalloc(const mt_bf16* dy, const mt_bf16* x, const mt_bf16* g, const float* rstd,
+                                            const mt_bf16* dres, mt_bf16* dx, float* dg, int64_t rows, int32_t H,
+                                            void* stream) {
+  if (!dy || !x || !g || !rstd || !dx || !dg) return fail(MT_ERR_INVALID_ARG, "rmsnorm_bwd_noalloc: NULL pointer");
+  if (rows < 0 || H <= 0 || H % 8)
+    return fail(MT_ERR_INVALID_ARG, "rmsnorm_bwd_noalloc: need rows >= 0, H > 0, H %% 8 == 0");
+  if (!aligned16(dy) || !aligned16(x) || !aligned16(g) || !aligned16(dx) || (dres && !aligned16(dres)))
+    return fail(MT_ERR_ALIGNMENT, "rmsnorm_bwd_noalloc: 16-byte alignment");
+  const uint64_t need = colsum_ws_bytes(rows, H);
+  if (need > static_cast<uint64_t>(NOALLOC_SCRATCH_FLOATS) * 4)
+    return fail(MT_ERR_WORKSPACE,
+                "rmsnorm_bwd_noalloc: %lld rows x %d columns need %llu bytes of scratch, above its fixed %lld bytes "
+                "(ceil(rows/64) * H must be <= %lld); use mt_rmsnorm_bwd with a workspace",
+                (long long)rows, H, (unsigned long long)need, (long long)(NOALLOC_SCRATCH_FLOATS * 4),
+                (long long)NOALLOC_SCRATCH_FLOATS);
+  float* scratch = nullptr;
+  MT_TRY(noalloc_scratch(&scratch));
+  return rmsnorm_bwd_launch(dy, x, g, rstd, dres, dx, dg, rows, H, scratch, as_stream(stream));
+}

@@ -161,6 +161,27 @@ mt_status mt_rmsnorm_bwd(const mt_bf16* dy, const mt_bf16* x, const mt_bf16* g, 
                          const mt_bf16* dres, mt_bf16* dx, float* dg, int64_t rows, int32_t H,
                          void* ws, uint64_t ws_bytes, void* stream);
 
+/* The same RMSNorm backward for callers that cannot allocate device memory:
+ * code whose device memory is owned and budgeted by another allocator (a
+ * framework's caching pool, a fixed budget reserved at start-up) and that has
+ * no spare buffer to hand over as workspace. It takes no workspace and calls
+ * no allocation routine; its scratch is a fixed 8 MiB array inside the library
+ * that every GPU which loads the library holds until the process exits. The
+ * MegaTrain pages have no counterpart: this is a calling convention only.
+ * - Limit: ceil(rows / 64) * H <= 2,097,152 (e.g. 32,768 rows of 3584, or
+ *   16,384 rows of 8192); larger calls return MT_ERR_WORKSPACE and change nothing.
+ * - The first call on each device looks up the array's device address with
+ *   that device current (cudaGetSymbolAddress); make that first call before
+ *   any stream capture.
+ * - All calls share the one array and it keeps the last call's contents. Every
+ *   partial sum a call reads it has written itself, so nothing needs clearing,
+ *   but calls that overlap on the GPU (different streams, or different host
+ *   threads without ordering) race on it: order them on one stream.
+ * Arguments and results are those of mt_rmsnorm_bwd; results are bitwise equal
+ * to it. */
+mt_status mt_rmsnorm_bwd_noalloc(const mt_bf16* dy, const mt_bf16* x, const mt_bf16* g, const float* rstd,
+                                 const mt_bf16* dres, mt_bf16* dx, float* dg, int64_t rows, int32_t H, void* stream);
+
 /* Rotate-half RoPE in place on the first n_heads heads (of head_dim d) of each
  * row of x (row stride ld elements; rows are [B, T], position = t). Pair
  * (i, i+d/2) rotates by t*theta^(-2i/d); inverse = 1 rotates by the negative

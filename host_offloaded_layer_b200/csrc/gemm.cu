@@ -24,7 +24,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
+#include <string>
 
 #include "mt_internal.h"
 
@@ -50,6 +52,7 @@ struct EpiArgs {
   int64_t ldc, ldr;
   int M, N, K;
   int c_f32, accumulate;
+  int raster;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -168,7 +171,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+// Output-tile order. raster 0: groups of 16 row-blocks, columns within a
+// group; raster 1: row-major over all column blocks (the B operand stays in
+// L2); raster 2: column-major over all row blocks (the A operand stays in L2).
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int& mb, int& nb) {
+  if (raster == 1) {
+    mb = t / num_n;
+    nb = t - mb * num_n;
+    return;
+  }
+  if (raster == 2) {
+    nb = t / num_m;
+    mb = t - nb * num_m;
+    return;
+  }
   constexpr int G = 16;
   const int group_tiles = G * num_n;
   const int g = t / group_tiles;
@@ -303,7 +319,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       int mb, nb;
-      tile_coords(t, num_m, num_n, mb, nb);
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       const int m0 = mb * BM, n0 = nb * BN;
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
@@ -394,7 +410,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int ab = tl & 1;
       const uint32_t aph = (tl >> 1) & 1u;
       int mb, nb;
-      tile_coords(t, num_m, num_n, mb, nb);
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + q * 32 + lane;
@@ -415,6 +431,264 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   fence_after();
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ============================================================== 2-SM kernel
+// The same contraction with tcgen05.mma.cta_group::2: a cluster of two CTAs
+// on two SMs computes a 256 x 256 output tile. Each CTA stages its own 128
+// rows of A and its own 128 columns' worth of B (6 stages of 32 KiB), so per
+// FLOP each SM moves a third less operand data through shared memory than the
+// one-SM 128 x 256 tile. The even CTA issues the MMAs for the pair; its full
+// barriers count both CTAs' TMA bytes, the MMA commits are multicast to both
+// CTAs' empty / accumulator-full barriers, and both CTAs' epilogue warps
+// arrive on the even CTA's accumulator-empty barrier. No TMA load uses
+// cluster multicast: every CTA loads its own operands.
+namespace c2 {
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+constexpr int HALF = 128 * BK * 2;  // 16 KiB: one CTA's A rows or B columns per stage
+constexpr int STAGE_BYTES = 2 * HALF;
+constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;
+}  // namespace c2
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load into this CTA's shared memory that completes its bytes on the
+// pair's barrier (which lives in the even CTA).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrives on the barrier at this shared offset in both CTAs of the pair once
+// the MMAs issued so far have completed.
+__device__ __forceinline__ void umma2_commit_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+__host__ __device__ constexpr uint32_t make_idesc2(bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(c2::BN >> 3) << 17) | (static_cast<uint32_t>(c2::BM >> 4) << 24);
+}
+
+// Bytes one CTA of the pair loads per stage (boxes wholly past M or N are skipped).
+__device__ __forceinline__ uint32_t half_bytes(bool a_mn, bool b_mn, int m0, int n0, int M, int N) {
+  uint32_t b = 0;
+  if (!a_mn) {
+    if (m0 < M) b += c2::HALF;
+  } else {
+    for (int j = 0; j < 2; ++j)
+      if (m0 + 64 * j < M) b += MN_BOX;
+  }
+  if (!b_mn) {
+    if (n0 < N) b += c2::HALF;
+  } else {
+    for (int j = 0; j < 2; ++j)
+      if (n0 + 64 * j < N) b += MN_BOX;
+  }
+  return b;
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, EpiArgs ep,
+                 int32_t* err) {
+  constexpr int BM = c2::BM, BN = c2::BN, BK = c2::BK, STAGES = c2::STAGES, HALF = c2::HALF;
+  constexpr int SMEM_TILES = c2::SMEM_TILES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * HALF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
+  uint64_t* full = bars;                // TMA (both CTAs) -> MMA; used in the even CTA
+  uint64_t* empty = bars + STAGES;      // MMA -> TMA, in each CTA
+  uint64_t* tfull = bars + 2 * STAGES;  // MMA -> epilogue, in each CTA
+  uint64_t* tempty = tfull + 2;         // epilogues of both CTAs -> MMA; used in the even CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int num_m = (ep.M + BM - 1) / BM, num_n = (ep.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (ep.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 2 * 128);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  cluster_sync();  // barriers of both CTAs are initialised before any remote use
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = cluster; t < num_tiles && ok; t += n_clusters) {
+      int mb, nb;
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      const int m_own = mb * BM + static_cast<int>(rank) * 128;  // this CTA's A rows
+      const int n_own = nb * BN + static_cast<int>(rank) * 128;  // this CTA's B rows
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!warp_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
+          if (rank == 0) {
+            const uint32_t bytes = half_bytes(A_MN, B_MN, mb * BM, nb * BN, ep.M, ep.N) +
+                                   half_bytes(A_MN, B_MN, mb * BM + 128, nb * BN + 128, ep.M, ep.N);
+            mbar_expect_tx(smem_u32(&full[s]), bytes);
+          }
+          const uint32_t a_dst = smem_u32(sA + s * HALF), b_dst = smem_u32(sB + s * HALF);
+          const int k0 = kb * BK;
+          if (!A_MN) {
+            if (m_own < ep.M) tma_load_2d_pair(a_dst, &tmA, fb, k0, m_own);
+          } else {
+            for (int j = 0; j < 2; ++j)
+              if (m_own + 64 * j < ep.M) tma_load_2d_pair(a_dst + j * MN_BOX, &tmA, fb, m_own + 64 * j, k0);
+          }
+          if (!B_MN) {
+            if (n_own < ep.N) tma_load_2d_pair(b_dst, &tmB, fb, k0, n_own);
+          } else {
+            for (int j = 0; j < 2; ++j)
+              if (n_own + 64 * j < ep.N) tma_load_2d_pair(b_dst + j * MN_BOX, &tmB, fb, n_own + 64 * j, k0);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    if (rank == 0) {
+      constexpr uint32_t idesc = make_idesc2(A_MN, B_MN);
+      uint32_t it = 0;
+      int tl = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += n_clusters, ++tl) {
+        const int ab = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1u;
+        if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
+        fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!warp_wait(smem_u32(&full[s]), ph, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          if (lane == 0) {
+            const uint32_t a_base = smem_u32(sA + s * HALF), b_base = smem_u32(sB + s * HALF);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad =
+                  A_MN ? smem_desc(a_base + kk * 2048, MN_BOX, 1024) : smem_desc(a_base + kk * 32, 16, 1024);
+              const uint64_t bd =
+                  B_MN ? smem_desc(b_base + kk * 2048, MN_BOX, 1024) : smem_desc(b_base + kk * 32, 16, 1024);
+              umma2_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma2_commit_both(smem_u32(&empty[s]));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) umma2_commit_both(smem_u32(&tfull[ab]));
+        __syncwarp();
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    int tl = 0;
+    for (int t = cluster; t < num_tiles; t += n_clusters, ++tl) {
+      const int ab = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1u;
+      int mb, nb;
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
+      fence_after();
+      const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        if (col0 >= ep.N) break;
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN + c * 32), r);
+        if (row < ep.M) store_chunk(ep, row, col0, r);
+      }
+      fence_before();
+      mbar_arrive_remote(map_to_rank(smem_u32(&tempty[ab]), 0));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still signal it
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
   }
 }
 
@@ -450,7 +724,7 @@ mt_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
 }
 
 template <bool A_MN, bool B_MN>
-mt_status launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
+mt_status launch_1sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -465,19 +739,80 @@ mt_status launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& 
   return launch_check("gemm_kernel");
 }
 
+// Largest number of 2-CTA clusters of gemm2_kernel that fit on the device at once.
+template <bool A_MN, bool B_MN>
+int max_pair_clusters() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = c2::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<A_MN, B_MN>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+template <bool A_MN, bool B_MN>
+mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err =
+        cudaFuncSetAttribute(gemm2_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, c2::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return fail(MT_ERR_CUDA, "gemm2 smem attribute: %s", cudaGetErrorString(attr_err));
+  const int num_tiles = ((ep.M + c2::BM - 1) / c2::BM) * ((ep.N + c2::BN - 1) / c2::BN);
+  const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN>());
+  int32_t* err = device_error_word();
+  if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
+  gemm2_kernel<A_MN, B_MN><<<2 * clusters, NUM_THREADS, c2::SMEM_BYTES, st>>>(ta, tb, ep, err);
+  return launch_check("gemm2_kernel");
+}
+
+// Which kernel runs: the 2-SM kernel unless MT_GEMM_KERNEL=1sm is set (kept for
+// comparison measurements).
+bool use_2sm() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MT_GEMM_KERNEL");
+    v = (e && std::string(e) == "1sm") ? 0 : 1;
+  }
+  return v == 1;
+}
+
+// Tile order that keeps the smaller operand resident in L2 when it fits.
+int pick_raster(int64_t M, int64_t N, int64_t K) {
+  const int64_t l2_budget = 40ll << 20;
+  if (N * K * 2 <= l2_budget) return 1;
+  if (M * K * 2 <= l2_budget) return 2;
+  return 0;
+}
+
 }  // namespace
 
 mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn, void* C,
                       int64_t ldc, bool c_f32, bool accumulate, int64_t M, int64_t N, int64_t K,
                       const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, cudaStream_t st) {
   if (M == 0 || N == 0) return MT_OK;
+  const bool two = use_2sm();
+  const uint32_t b_rows = two ? 128 : BN;  // rows of a K-major B box
   CUtensorMap ta, tb;
   if (!a_mn)
-    MT_TRY(make_map(&ta, A, K, M, lda, 64, BM));
+    MT_TRY(make_map(&ta, A, K, M, lda, 64, 128));
   else
     MT_TRY(make_map(&ta, A, M, K, lda, 64, 64));
   if (!b_mn)
-    MT_TRY(make_map(&tb, B, K, N, ldb, 64, BN));
+    MT_TRY(make_map(&tb, B, K, N, ldb, 64, b_rows));
   else
     MT_TRY(make_map(&tb, B, N, K, ldb, 64, 64));
   EpiArgs ep;
@@ -491,18 +826,30 @@ mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B
   ep.K = static_cast<int>(K);
   ep.c_f32 = c_f32 ? 1 : 0;
   ep.accumulate = accumulate ? 1 : 0;
+  ep.raster = pick_raster(M, N, K);
   const double flops = 2.0 * double(M) * double(N) * double(K);
   GemmTimer* tm = current_gemm_timer();
   if (tm) tm->before(st);
   mt_status s;
-  if (!a_mn && !b_mn)
-    s = launch_t<false, false>(ta, tb, ep, st);
-  else if (!a_mn && b_mn)
-    s = launch_t<false, true>(ta, tb, ep, st);
-  else if (a_mn && !b_mn)
-    s = launch_t<true, false>(ta, tb, ep, st);
-  else
-    s = launch_t<true, true>(ta, tb, ep, st);
+  if (two) {
+    if (!a_mn && !b_mn)
+      s = launch_2sm<false, false>(ta, tb, ep, st);
+    else if (!a_mn && b_mn)
+      s = launch_2sm<false, true>(ta, tb, ep, st);
+    else if (a_mn && !b_mn)
+      s = launch_2sm<true, false>(ta, tb, ep, st);
+    else
+      s = launch_2sm<true, true>(ta, tb, ep, st);
+  } else {
+    if (!a_mn && !b_mn)
+      s = launch_1sm<false, false>(ta, tb, ep, st);
+    else if (!a_mn && b_mn)
+      s = launch_1sm<false, true>(ta, tb, ep, st);
+    else if (a_mn && !b_mn)
+      s = launch_1sm<true, false>(ta, tb, ep, st);
+    else
+      s = launch_1sm<true, true>(ta, tb, ep, st);
+  }
   if (tm) tm->after(st, flops);
   add_exec_flops(flops);
   return s;

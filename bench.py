@@ -68,6 +68,21 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The slowest rank's time (all ranks call this in the same order)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time (per second)."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def model_flops(cfg, p_layer):
     sh = cfg["shape"]
     return metrics.model_flops(cfg["L"] * p_layer, cfg["L"], sh["hidden"], cfg["B"], cfg["T"])
@@ -271,11 +286,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             fn()
         ev1.record(cs)
         barrier()
-        ms = ev0.elapsed_time(ev1)
-        if pg is not None:
-            t = torch.tensor([ms], device="cuda")
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
         return ms / steps
 
     dev_step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d, c_sink)  # noqa: E731
@@ -295,8 +306,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     link = measure_link(torch) if rank == 0 else None
 
     mflops = model_flops(cfg, p_layer)
-    value = mflops * world / (ms / 1e3) / 1e12
-    e2e = mflops * world / (ms_e2e / 1e3) / 1e12
+    value = job_throughput(mflops, world, ms) / 1e12
+    e2e = job_throughput(mflops, world, ms_e2e) / 1e12
     peaks, src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     gemm_tf = st.gemm_flops / (st.gemm_ms / 1e3) / 1e12 if st.gemm_ms > 0 else None

@@ -51,6 +51,13 @@ CONFIGS = {
     4: dict(name="qwen2.5-14b-shape_x48_b64x1024", shape=QWEN14B, L=48, B=64, T=1024, K=4, chunk=0),
     5: dict(name="qwen2.5-7b-shape_x28_b1x32768_mlpchunk4096", shape=QWEN7B, L=28, B=1, T=32768, K=4, chunk=4096),
 }
+# The ablations of MegaTrain Table 4, as engine options.
+ABLATIONS = {
+    "none": {},
+    "single_buffer": {"n_weight_slots": 1},  # "w/o Double Buffering"
+    "no_slab_pool": {"no_slab_pool": 1},     # "w/o Gradient Slab Pool"
+    "ckpt1": {"ckpt_interval": 1},           # "w/ Checkpoint Interval=1"
+}
 METRIC = "sustained TFLOPS (6ND+12LHT²) & tokens/s, streamed 7B/14B layer stack, 1 B200"
 UNIT = "TFLOPS"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -249,7 +256,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     lcfg = L_.make_cfg(**sh)
     p_layer = L_.mt_layer_param_count(lcfg)
     nL, B, T = cfg["L"], cfg["B"], cfg["T"]
-    opts = L_.make_opts(ckpt_interval=cfg["K"], mlp_chunk=cfg["chunk"], time_gemms=1, timeout_ms=120000)
+    abl = ABLATIONS[args.ablation]
+    opts = L_.make_opts(ckpt_interval=abl.get("ckpt_interval", cfg["K"]), mlp_chunk=cfg["chunk"], time_gemms=1,
+                        timeout_ms=120000, n_weight_slots=abl.get("n_weight_slots", 0),
+                        no_slab_pool=abl.get("no_slab_pool", 0))
     store = L_.mt_host_store_create(lcfg, nL, True)
     fill_store(L_, store, lcfg, nL)
     nbytes = L_.mt_engine_workspace_bytes(lcfg, nL, B, T, opts)
@@ -324,7 +334,8 @@ def run_ours(args, cfg, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": cfg["name"], "layers": nL, "batch": B, "seq_len": T, "ckpt_interval": cfg["K"],
+            "config": {"workload": cfg["name"], "layers": nL, "batch": B, "seq_len": T,
+                       "ckpt_interval": abl.get("ckpt_interval", cfg["K"]), "ablation": args.ablation,
                        "mlp_chunk": cfg["chunk"], "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each layer's weights alone are %.0f MB)" % (p_layer * 2 / 1e6),
                        "sink": "pinned slab handed to a no-op host callback"},
@@ -363,6 +374,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ablation", default="none", choices=sorted(ABLATIONS),
+                    help="engine variant of MegaTrain Table 4 (default: the full system)")
     args = ap.parse_args()
     rank, world, local_rank = dist_env()
     cfg = CONFIGS[args.config]

@@ -43,7 +43,8 @@ class mt_param_offsets(ctypes.Structure):
 
 class mt_engine_opts(ctypes.Structure):
     _fields_ = [(n, c_i32) for n in ("ckpt_interval", "n_weight_slots", "n_host_slabs", "n_dev_grad_slabs",
-                                     "mlp_chunk", "resident", "timeout_ms", "fail_h2d_at", "time_gemms")]
+                                     "mlp_chunk", "resident", "timeout_ms", "fail_h2d_at", "time_gemms",
+                                     "no_slab_pool")]
 
 
 class mt_stats(ctypes.Structure):
@@ -69,6 +70,7 @@ _SIGS = {
     "mt_layer_recompute_bwd": (c_i32, [_CFG, _P, _P, _P, _P, _P, c_i32, c_i32, c_i32, _P, c_u64, _P]),
     "mt_gemm_bf16": (c_i32, [_P, c_i64, c_i32, _P, c_i64, c_i32, _P, c_i64, c_i32, c_i32, c_i64, c_i64, c_i64,
                              _P, _P, c_i64, _P]),
+    "mt_gemm_swiglu_bf16": (c_i32, [_P, c_i64, _P, c_i64, _P, c_i64, _P, c_i64, c_i64, c_i64, c_i64, _P]),
     "mt_rmsnorm_fwd": (c_i32, [_P, _P, _P, _P, c_i64, c_i32, c_f32, _P]),
     "mt_rmsnorm_bwd_workspace_bytes": (c_u64, [c_i64, c_i32]),
     "mt_rmsnorm_bwd": (c_i32, [_P, _P, _P, _P, _P, _P, _P, c_i64, c_i32, _P, c_u64, _P]),
@@ -189,6 +191,11 @@ def mt_gemm_bf16(A, lda, a_mn_major, Bm, ldb, b_mn_major, C, ldc, c_f32, accumul
                                M, N, K, _ptr(bias), _ptr(residual), ldr, _stream(stream)))
 
 
+def mt_gemm_swiglu_bf16(A, lda, Wgu, ldw, m, ldm, gu, ld_gu, M, F, K, stream=None):
+    _check(load().mt_gemm_swiglu_bf16(_ptr(A), lda, _ptr(Wgu), ldw, _ptr(m), ldm, _ptr(gu), ld_gu, M, F, K,
+                                      _stream(stream)))
+
+
 def mt_rmsnorm_fwd(x, g, y, rstd, rows, H, eps, stream=None):
     _check(load().mt_rmsnorm_fwd(_ptr(x), _ptr(g), _ptr(y), _ptr(rstd), rows, H, eps, _stream(stream)))
 
@@ -263,9 +270,9 @@ def mt_host_store_destroy(store):
 
 
 def make_opts(ckpt_interval=4, n_weight_slots=0, n_host_slabs=0, n_dev_grad_slabs=0, mlp_chunk=0, resident=0,
-              timeout_ms=0, fail_h2d_at=0, time_gemms=0) -> mt_engine_opts:
+              timeout_ms=0, fail_h2d_at=0, time_gemms=0, no_slab_pool=0) -> mt_engine_opts:
     return mt_engine_opts(ckpt_interval, n_weight_slots, n_host_slabs, n_dev_grad_slabs, mlp_chunk, resident,
-                          timeout_ms, fail_h2d_at, time_gemms)
+                          timeout_ms, fail_h2d_at, time_gemms, no_slab_pool)
 
 
 def mt_engine_workspace_bytes(cfg, n_layers, B, T, opts) -> int:

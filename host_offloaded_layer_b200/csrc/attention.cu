@@ -10,7 +10,9 @@
 // (looping over key blocks), another computes dK and dV per key block,
 // looping over the query heads of its group in a fixed order and over the
 // query blocks at or after the diagonal. No atomics are used.
+#include <cstdlib>
 #include <mutex>
+#include <string>
 
 #include "mt_internal.h"
 
@@ -666,9 +668,24 @@ uint64_t attn_bwd_ws_bytes(int B, int T, int nq) {
   return static_cast<uint64_t>(align_up(static_cast<int64_t>(B) * nq * T * 4, 256));
 }
 
+mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T,
+                             int nq, int nkv, cudaStream_t st);
+
+// head_dim 128 runs the tcgen05 forward unless MT_ATTN_FWD=mma is set (kept for
+// comparison measurements); head_dim 64 runs the mma.sync forward.
+static bool use_tc_fwd() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MT_ATTN_FWD");
+    v = (e && std::string(e) == "mma") ? 0 : 1;
+  }
+  return v == 1;
+}
+
 mt_status attn_fwd_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T, int nq,
                           int nkv, int d, cudaStream_t st) {
   if (B == 0 || T == 0) return MT_OK;
+  if (d == 128 && use_tc_fwd()) return attn_fwd_tc_launch(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
   if (d == 128) return fwd_t<128>(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
   if (d == 64) return fwd_t<64>(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
   return fail(MT_ERR_UNSUPPORTED, "attention supports head_dim 64 and 128, not %d", d);

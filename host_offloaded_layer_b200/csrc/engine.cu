@@ -169,7 +169,8 @@ struct EventTimer : GemmTimer {
 };
 
 struct SinkItem {
-  int jb, layer, slab;
+  int jb, layer, slab;  // slab: pool index, or -1 for a record pinned for this layer only
+  float* ptr;
 };
 
 }  // namespace
@@ -221,6 +222,7 @@ mt_status validate_opts(const mt_engine_opts* in, int L, mt_engine_opts* o) {
   if (!in) return fail(MT_ERR_INVALID_ARG, "opts is NULL");
   *o = *in;
   if (o->ckpt_interval < 1) return fail(MT_ERR_INVALID_ARG, "ckpt_interval must be >= 1");
+  if (o->no_slab_pool < 0) return fail(MT_ERR_INVALID_ARG, "no_slab_pool must be 0 or 1");
   if (o->n_weight_slots < 0 || o->n_host_slabs < 0 || o->n_dev_grad_slabs < 0 || o->mlp_chunk < 0 ||
       o->timeout_ms < 0 || o->fail_h2d_at < 0)
     return fail(MT_ERR_INVALID_ARG, "engine options must be >= 0");
@@ -305,12 +307,13 @@ void sink_loop(mt_engine* e, mt_grad_sink sink, void* user) {
     mt_status s = poll_event(e->d2h_done[it.jb], deadline, "gradient offload");
     if (s == MT_OK && sink) {
       const auto t0 = Clock::now();
-      int32_t rc = sink(it.layer, e->slab[it.slab], rec, user);
+      int32_t rc = sink(it.layer, it.ptr, rec, user);
       e->st.sink_ms += std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
       if (rc != 0) s = fail(MT_ERR_SINK, "gradient sink returned %d for layer %d", rc, it.layer);
     }
+    if (it.slab < 0) cudaFreeHost(it.ptr);  // no pool: the record was pinned for this layer only
     std::lock_guard<std::mutex> lk(e->mu);
-    e->free_slabs.push_back(it.slab);
+    if (it.slab >= 0) e->free_slabs.push_back(it.slab);
     if (s != MT_OK) {
       e->sink_status = s;
       e->abort = true;
@@ -359,7 +362,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
     e->sink_status = MT_OK;
     e->sink_finished = false;
     e->free_slabs.clear();
-    for (int i = 0; i < e->NS; ++i) e->free_slabs.push_back(i);
+    for (int i = 0; i < static_cast<int>(e->slab.size()); ++i) e->free_slabs.push_back(i);
   }
   if (e->sink_thread.joinable()) e->sink_thread.join();  // finished: checked by the caller
   e->sink_thread = std::thread(sink_loop, e, sink, user);
@@ -434,9 +437,16 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       e->st.layer_bwd_calls++;
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
       if (status == MT_OK) {
-        // take a pinned slab from the pool (bounded wait), then offload
+        // take a pinned slab from the pool (bounded wait), then offload. Without the pool
+        // (the Table 4 ablation) a record is pinned for this layer and freed after its sink.
         int p = -1;
-        {
+        float* dst = nullptr;
+        if (e->opts.no_slab_pool) {
+          if (cudaHostAlloc(reinterpret_cast<void**>(&dst), rec * 4, cudaHostAllocPortable) != cudaSuccess) {
+            cudaGetLastError();
+            status = fail(MT_ERR_OOM, "pinned allocation of a gradient record failed");
+          }
+        } else {
           std::unique_lock<std::mutex> lk(e->mu);
           const bool got = e->cv.wait_for(lk, timeout, [e] { return !e->free_slabs.empty() || e->abort; });
           if (e->abort) {
@@ -446,6 +456,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
           } else {
             p = e->free_slabs.back();
             e->free_slabs.pop_back();
+            dst = e->slab[p];
           }
         }
         // two pieces: the MLP weights' gradients (the record's tail from Wg on) as soon as
@@ -453,22 +464,25 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         const uint64_t split = e->G.off.wg;
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->mlp_done[jb], 0), "wait mlp_done");
         if (status == MT_OK)
-          status = cuda_check(cudaMemcpyAsync(e->slab[p] + split, e->dgrad[ns] + split, (rec - split) * 4,
+          status = cuda_check(cudaMemcpyAsync(dst + split, e->dgrad[ns] + split, (rec - split) * 4,
                                               cudaMemcpyDeviceToHost, e->os),
                               "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->g_ready[jb], 0), "wait g_ready");
         if (status == MT_OK)
           status = cuda_check(
-              cudaMemcpyAsync(e->slab[p], e->dgrad[ns], split * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
+              cudaMemcpyAsync(dst, e->dgrad[ns], split * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaEventRecord(e->d2h_done[jb], e->os), "record d2h_done");
         if (status == MT_OK) {
           e->st.d2h_bytes += rec * 4;
           std::lock_guard<std::mutex> lk(e->mu);
-          e->queue.push_back({jb, l, p});
+          e->queue.push_back({jb, l, p, dst});
           e->cv.notify_all();
         } else if (p >= 0) {
           std::lock_guard<std::mutex> lk(e->mu);
           e->free_slabs.push_back(p);
+        } else if (dst) {
+          cudaStreamSynchronize(e->os);
+          cudaFreeHost(dst);
         }
       }
       ++jb;
@@ -557,7 +571,7 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
     return s;
   };
   const uint64_t rec = G.off.record_elems;
-  for (int i = 0; i < e->NS; ++i) {
+  for (int i = 0; i < (o.no_slab_pool ? 0 : e->NS); ++i) {
     float* p = nullptr;
     if (cudaHostAlloc(reinterpret_cast<void**>(&p), rec * 4, cudaHostAllocPortable) != cudaSuccess) {
       cudaGetLastError();
@@ -671,6 +685,8 @@ mt_status mt_engine_reset(mt_engine* e) {
   MT_TRY(poll_stream(e->os, deadline, "offload stream"));
   std::lock_guard<std::mutex> lk(e->mu);
   e->abort = false;
+  for (const SinkItem& it : e->queue)
+    if (it.slab < 0) cudaFreeHost(it.ptr);
   e->queue.clear();
   e->sink_status = MT_OK;
   return MT_OK;

@@ -34,6 +34,9 @@ mt_status attn_fwd_launch(const mt_bf16*, int64_t, mt_bf16*, int64_t, float*, in
 mt_status attn_bwd_launch(const mt_bf16*, int64_t, const mt_bf16*, const mt_bf16*, int64_t, const float*, mt_bf16*,
                           int, int, int, int, int, void*, cudaStream_t);
 uint64_t attn_bwd_ws_bytes(int B, int T, int nq);
+bool gemm_swiglu_available();
+mt_status gemm_swiglu_launch(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m, int64_t ldm,
+                             mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st);
 
 namespace {
 
@@ -96,10 +99,15 @@ mt_status attention_half(const Geom& G, const mt_bf16* w, const mt_bf16* x, int 
   return MT_OK;
 }
 
-// [g|u] = h2c Wgu^T; m = silu(g) * u for one chunk of rows.
-mt_status mlp_up(const Geom& G, const mt_bf16* w, const mt_bf16* h2c, int64_t rows, const LayerWs& ws,
+// [g|u] = h2c Wgu^T; m = silu(g) * u for one chunk of rows. With the 2-SM GEMM
+// the SwiGLU is its epilogue (m from the fp32 accumulators; g and u are only
+// written when the backward needs them); otherwise a separate pass.
+mt_status mlp_up(const Geom& G, const mt_bf16* w, const mt_bf16* h2c, int64_t rows, const LayerWs& ws, bool need_gu,
                  cudaStream_t st) {
   const mt_param_offsets& O = G.off;
+  if (gemm_swiglu_available())
+    return gemm_swiglu_launch(h2c, G.H, w + O.wg, G.H, ws.m, G.F, need_gu ? ws.gu : nullptr, 2 * G.F, rows, G.F, G.H,
+                              st);
   MT_TRY(gemm_launch(h2c, G.H, false, w + O.wg, G.H, false, ws.gu, 2 * G.F, false, false, rows, 2 * G.F, G.H, nullptr,
                      nullptr, 0, st));
   MT_TRY(swiglu_fwd_launch(ws.gu, ws.m, rows, static_cast<int>(G.F), st));
@@ -140,7 +148,7 @@ mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_b
   const mt_param_offsets& O = G.off;
   for (int64_t r0 = 0; r0 < M; r0 += Mc) {
     const int64_t rows = std::min(Mc, M - r0);
-    MT_TRY(mlp_up(G, w_dev, w.h2 + r0 * G.H, rows, w, st));
+    MT_TRY(mlp_up(G, w_dev, w.h2 + r0 * G.H, rows, w, false, st));
     MT_TRY(gemm_launch(w.m, G.F, false, w_dev + O.wd, G.F, false, y + r0 * G.H, G.H, false, false, rows, G.H, G.F,
                        nullptr, w.x2 + r0 * G.H, G.H, st));
   }
@@ -187,7 +195,7 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
     const bool acc = r0 > 0;
     const mt_bf16* h2c = w.h2 + r0 * G.H;
     const mt_bf16* dyc = dy + r0 * G.H;
-    MT_TRY(mlp_up(G, w_dev, h2c, rows, w, st));
+    MT_TRY(mlp_up(G, w_dev, h2c, rows, w, true, st));
     // dWd (+)= dy^T m
     MT_TRY(gemm_launch(dyc, G.H, true, w.m, G.F, true, dw_dev + O.wd, G.F, true, acc, G.H, G.F, rows, nullptr, nullptr,
                        0, st));

@@ -146,6 +146,16 @@ mt_status mt_gemm_bf16(const mt_bf16* A, int64_t lda, int32_t a_mn_major,
                        int64_t M, int64_t N, int64_t K,
                        const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, void* stream);
 
+/* The gate/up projection with the SwiGLU activation as its epilogue (2-SM
+ * tcgen05 kernel). Wgu is [2F, K] (Wg rows then Wu rows, K-major), A is [M, K]
+ * K-major. m[r, j] = silu(g) * u with g = A_r . Wg_j and u = A_r . Wu_j taken
+ * from the fp32 accumulators; when gu is not NULL, g and u are also stored
+ * (bf16) to gu[r, j] and gu[r, F + j]. Pointers 16-byte aligned; lda, ldw,
+ * ldm, ld_gu and F multiples of 8. MT_ERR_UNSUPPORTED when the library runs
+ * its one-SM GEMM kernel (MT_GEMM_KERNEL=1sm). */
+mt_status mt_gemm_swiglu_bf16(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m,
+                              int64_t ldm, mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, void* stream);
+
 /* RMSNorm forward over rows of H: y = x * rstd * g, rstd = 1/sqrt(mean x^2 + eps)
  * (fp32 [rows] out). */
 mt_status mt_rmsnorm_fwd(const mt_bf16* x, const mt_bf16* g, mt_bf16* y, float* rstd,
@@ -257,6 +267,8 @@ typedef struct mt_engine_opts {
   int32_t timeout_ms;      /* bound of every host wait (0 = 60000) */
   int32_t fail_h2d_at;     /* fault injection: the n-th weight copy fails (0 = off) */
   int32_t time_gemms;      /* 1: time every GEMM launch with CUDA events (stats) */
+  int32_t no_slab_pool;    /* 1: pin a gradient record per layer and free it after its sink
+                              (the "w/o Gradient Slab Pool" ablation of MegaTrain Table 4) */
 } mt_engine_opts;
 
 /* Gradient sink: called on a library thread, in backward order, with layer l's

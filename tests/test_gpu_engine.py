@@ -102,7 +102,7 @@ def test_streamed_step_matches_oracle(n_layers, K):
 def test_streamed_schedules_are_bit_exact_to_resident():
     runs = {}
     for name, opts in {"resident": dict(resident=1), "double": dict(), "single": dict(n_weight_slots=1),
-                       "pool1": dict(n_host_slabs=1, n_dev_grad_slabs=1)}.items():
+                       "pool1": dict(n_host_slabs=1, n_dev_grad_slabs=1), "nopool": dict(no_slab_pool=1)}.items():
         s = Stack(TINY, 5, 2, 128, ckpt_interval=2, **opts)
         try:
             y, dx, g = s.step()

@@ -80,6 +80,29 @@ def test_gemm_is_deterministic_and_covers_many_waves():
     _check_dev_error()
 
 
+@pytest.mark.parametrize("M,F,K", [(256, 688, 256), (200, 1000, 136), (8192, 18944, 3584)])
+def test_gemm_with_swiglu_epilogue(M, F, K):
+    import torch
+    A = _bits(9, 1, M * K, 1.0).reshape(M, K)
+    W = _bits(9, 2, 2 * F * K, 0.05).reshape(2 * F, K)
+    m = torch.zeros(M, F, dtype=torch.bfloat16, device="cuda")
+    gu = torch.zeros(M, 2 * F, dtype=torch.bfloat16, device="cuda")
+    L.mt_gemm_swiglu_bf16(H.dev_bf16(A), K, H.dev_bf16(W), K, m, F, gu, 2 * F, M, F, K)
+    torch.cuda.synchronize()
+    _check_dev_error()
+    rows = np.arange(M) if M <= 256 else np.random.default_rng(0).choice(M, 96, replace=False)
+    a64 = H.bits_to_f64(A)[rows]
+    w64 = H.bits_to_f64(W)
+    g, u = a64 @ w64[:F].T, a64 @ w64[F:].T
+    assert H.rel(H.host_f64(m)[rows], O.swiglu_fwd(g, u)) < 1e-2
+    got = H.host_f64(gu)[rows]
+    assert H.rel(got[:, :F], g) < 1e-2 and H.rel(got[:, F:], u) < 1e-2
+    m2 = torch.zeros_like(m)  # without g, u
+    L.mt_gemm_swiglu_bf16(H.dev_bf16(A), K, H.dev_bf16(W), K, m2, F, None, 0, M, F, K)
+    torch.cuda.synchronize()
+    assert torch.equal(m.view(torch.int16), m2.view(torch.int16))
+
+
 # ------------------------------------------------------------------ RMSNorm
 @pytest.mark.parametrize("rows,Hd", [(256, 256), (1000, 3584), (37, 5120)])
 def test_rmsnorm_forward_and_backward(rows, Hd):
@@ -170,6 +193,8 @@ ATTN_CASES = [
     (1, 200, 7, 1, 128),    # ragged, group of 7 (the 7B ratio)
     (1, 320, 28, 4, 128),   # 7B heads
     (2, 64, 2, 1, 128),
+    (2, 1024, 28, 4, 128),  # the 7B heads over 8 key blocks (online-softmax rescaling)
+    (2, 700, 8, 2, 128),    # ragged last query block that reaches into the next sequence and past the end
 ]
 
 

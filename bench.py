@@ -281,6 +281,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         return 0
 
     c_sink = L_.mt_grad_sink(sink)
+    sink_user = None
+    opt = None
+    if args.sink == "adamw":  # the library's CPU AdamW: a full training step including the optimizer
+        opt = L_.mt_host_optimizer_create(store, L_.mt_adamw_cfg(1e-5, 0.9, 0.95, 1e-8, 0.01, 0))
+        c_sink, sink_user = L_.optimizer_sink(), opt
     cs = streams[0]
 
     def barrier():
@@ -299,8 +304,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         ms = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
         return ms / steps
 
-    dev_step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d, c_sink)  # noqa: E731
-    host_step = lambda: L_.mt_stream_step_host(eng, store, xh, dyh, yh, dxh, c_sink)  # noqa: E731
+    dev_step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d, c_sink, sink_user)  # noqa: E731
+    host_step = lambda: L_.mt_stream_step_host(eng, store, xh, dyh, yh, dxh, c_sink, sink_user)  # noqa: E731
     for _ in range(args.warmup):
         dev_step()
     clocks = ClockSampler(local_rank)
@@ -338,7 +343,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                        "ckpt_interval": abl.get("ckpt_interval", cfg["K"]), "ablation": args.ablation,
                        "mlp_chunk": cfg["chunk"], "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each layer's weights alone are %.0f MB)" % (p_layer * 2 / 1e6),
-                       "sink": "pinned slab handed to a no-op host callback"},
+                       "sink": ("CPU AdamW on the fp32 master + bf16 refresh (library sink)" if args.sink == "adamw"
+                                else "pinned slab handed to a no-op host callback")},
             "tokens_per_s": B * T * world / (ms / 1e3),
             "clocks": clk,
             "e2e": {"value": e2e, "unit": UNIT,
@@ -359,6 +365,8 @@ def run_ours(args, cfg, rank, world, local_rank):
             "device_workspace_gb": nbytes / 1e9,
         }
     L_.mt_engine_destroy(eng)
+    if opt is not None:
+        L_.mt_host_optimizer_destroy(opt)
     L_.mt_host_store_destroy(store)
     if pg is not None:
         pg.barrier()
@@ -374,6 +382,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sink", default="none", choices=["none", "adamw"],
+                    help="what receives each layer's gradient record (adamw: the CPU optimizer step)")
     ap.add_argument("--ablation", default="none", choices=sorted(ABLATIONS),
                     help="engine variant of MegaTrain Table 4 (default: the full system)")
     args = ap.parse_args()

@@ -55,6 +55,11 @@ class mt_stats(ctypes.Structure):
                 ("sink_ms", ctypes.c_double), ("kernel_launches", c_u64)]
 
 
+class mt_adamw_cfg(ctypes.Structure):
+    _fields_ = [("lr", c_f32), ("beta1", c_f32), ("beta2", c_f32), ("eps", c_f32), ("weight_decay", c_f32),
+                ("n_threads", c_i32)]
+
+
 mt_grad_sink = ctypes.CFUNCTYPE(c_i32, c_i32, ctypes.POINTER(c_f32), c_u64, c_vp)
 
 _P = c_vp
@@ -97,6 +102,10 @@ _SIGS = {
     "mt_engine_stats": (c_i32, [c_vp, ctypes.POINTER(mt_stats)]),
     "mt_engine_reset": (c_i32, [c_vp]),
     "mt_engine_destroy": (None, [c_vp]),
+    "mt_adamw_update": (c_i32, [_P, _P, _P, _P, c_u64, ctypes.POINTER(mt_adamw_cfg), c_i64]),
+    "mt_host_optimizer_create": (c_i32, [c_vp, ctypes.POINTER(mt_adamw_cfg), ctypes.POINTER(c_vp)]),
+    "mt_host_optimizer_sink": (c_i32, [c_i32, ctypes.POINTER(c_f32), c_u64, c_vp]),
+    "mt_host_optimizer_destroy": (None, [c_vp]),
     "mt_schedule_len": (c_i32, [c_i32, c_i32]),
     "mt_schedule": (c_i32, [c_i32, c_i32, c_i32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32),
                             ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
@@ -318,3 +327,22 @@ def mt_schedule(n_layers, K, n_slots):
     arrs = [(c_i32 * n)() for _ in range(4)]
     _check(load().mt_schedule(n_layers, K, n_slots, *arrs))
     return [list(a) for a in arrs]
+
+
+def mt_adamw_update(w, m, v, g, n, cfg, t):
+    _check(load().mt_adamw_update(_ptr(w), _ptr(m), _ptr(v), _ptr(g), n, ctypes.byref(cfg), t))
+
+
+def mt_host_optimizer_create(store, cfg) -> int:
+    h = c_vp()
+    _check(load().mt_host_optimizer_create(store, ctypes.byref(cfg), ctypes.byref(h)))
+    return h.value
+
+
+def mt_host_optimizer_destroy(opt):
+    load().mt_host_optimizer_destroy(opt)
+
+
+def optimizer_sink():
+    """The library's AdamW sink as a callable for mt_stream_step (pass the optimizer as `user`)."""
+    return ctypes.cast(load().mt_host_optimizer_sink, mt_grad_sink)

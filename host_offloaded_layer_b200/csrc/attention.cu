@@ -17,6 +17,10 @@
 #include "mt_internal.h"
 
 namespace mt {
+
+mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o, int64_t ld_o, const float* lse,
+                             const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, cudaStream_t st);
+
 namespace {
 
 constexpr float LOG2E = 1.4426950408889634f;
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NT, 1)
   float* sL = reinterpret_cast<float*>(smem + 6 * C::TILE);  // [2][64] lse (log2 domain)
   float* sD = sL + 2 * 64;                                   // [2][64] delta
 
-  const int kb = gridDim.x - 1 - blockIdx.x;
+  const int kb = blockIdx.x;  // small key blocks have the most query blocks: first
   const int c = blockIdx.y, b = blockIdx.z;
   const int grp = nq / nkv;
   const int k0 = kb * C::BKV;
@@ -627,6 +631,17 @@ mt_status fwd_t(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float*
   return MT_OK;
 }
 
+// head_dim 128 runs the tcgen05 backward unless MT_ATTN_BWD=mma is set (kept for
+// comparison measurements).
+bool use_tc_bwd() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MT_ATTN_BWD");
+    v = (e && std::string(e) == "mma") ? 0 : 1;
+  }
+  return v == 1;
+}
+
 template <int D>
 mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16* d_o, int64_t ld_o, const float* lse,
                 mt_bf16* dqkv, int B, int T, int nq, int nkv, float* delta, cudaStream_t st) {
@@ -643,6 +658,7 @@ mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16*
   attn_delta_kernel<D><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, delta, rows, T, nq);
   MT_TRY(launch_check("attn_delta_kernel"));
+  if (D == 128 && use_tc_bwd()) return attn_bwd_tc_launch(qkv, ld, d_o, ld_o, lse, delta, dqkv, B, T, nq, nkv, st);
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
   const float scale_log2 = LOG2E * scale;
   dim3 gq((T + C::BQ - 1) / C::BQ, nq, B);

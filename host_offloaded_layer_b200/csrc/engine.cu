@@ -21,6 +21,8 @@
 // the engine's timeout; nothing waits on the device.
 #include <atomic>
 #include <chrono>
+#include <cmath>
+#include <cstdlib>
 #include <condition_variable>
 #include <cstring>
 #include <deque>
@@ -710,6 +712,127 @@ void mt_engine_destroy(mt_engine* e) {
   if (e->fin) cudaEventDestroy(e->fin);
   for (float* p : e->slab) cudaFreeHost(p);
   delete e;
+}
+
+}  // extern "C"
+
+// ======================================================================= CPU optimizer
+// The optimizer step of the memory-centric design runs on the host (blog
+// summary, design point 1: "Optimizer steps execute entirely on the CPU",
+// with Adam momentum and variance in host memory). AdamW (decoupled weight
+// decay): m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+// w -= lr * (m / (1-b1^t) / (sqrt(v / (1-b2^t)) + eps) + wd * w).
+struct mt_host_optimizer {
+  mt_host_store* store;
+  mt_adamw_cfg cfg;
+  float* m = nullptr;
+  float* v = nullptr;
+  std::vector<int64_t> steps;  // per layer: updates applied so far
+};
+
+static mt_status adamw_check(const mt_adamw_cfg* c) {
+  if (!c) return fail(MT_ERR_INVALID_ARG, "adamw cfg is NULL");
+  if (!(c->lr >= 0.f) || !(c->beta1 >= 0.f && c->beta1 < 1.f) || !(c->beta2 >= 0.f && c->beta2 < 1.f) ||
+      !(c->eps > 0.f) || !(c->weight_decay >= 0.f))
+    return fail(MT_ERR_INVALID_ARG, "adamw: need lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
+  return MT_OK;
+}
+
+static void adamw_range(float* w, float* m, float* v, const float* g, int64_t a, int64_t b, const mt_adamw_cfg& c,
+                        double bc1, double bc2) {
+  const float b1 = c.beta1, b2 = c.beta2, lr = c.lr, eps = c.eps, wd = c.weight_decay;
+  const float ib1 = static_cast<float>(1.0 / bc1), ib2 = static_cast<float>(1.0 / bc2);
+  for (int64_t i = a; i < b; ++i) {
+    const float gi = g[i];
+    const float mi = b1 * m[i] + (1.f - b1) * gi;
+    const float vi = b2 * v[i] + (1.f - b2) * gi * gi;
+    m[i] = mi;
+    v[i] = vi;
+    w[i] -= lr * ((mi * ib1) / (std::sqrt(vi * ib2) + eps) + wd * w[i]);
+  }
+}
+
+extern "C" {
+
+mt_status mt_adamw_update(float* w, float* m, float* v, const float* g, uint64_t n, const mt_adamw_cfg* cfg,
+                          int64_t t) {
+  MT_TRY(adamw_check(cfg));
+  if (!w || !m || !v || !g) return fail(MT_ERR_INVALID_ARG, "adamw: NULL array");
+  if (t < 1) return fail(MT_ERR_INVALID_ARG, "adamw: step t must be >= 1");
+  const double bc1 = 1.0 - std::pow(static_cast<double>(cfg->beta1), static_cast<double>(t));
+  const double bc2 = 1.0 - std::pow(static_cast<double>(cfg->beta2), static_cast<double>(t));
+  const mt_adamw_cfg c = *cfg;
+  parallel_for(static_cast<int64_t>(n), cfg->n_threads > 0 ? cfg->n_threads : default_threads(),
+               [&](int64_t a, int64_t b) { adamw_range(w, m, v, g, a, b, c, bc1, bc2); });
+  return MT_OK;
+}
+
+mt_status mt_host_optimizer_create(mt_host_store* store, const mt_adamw_cfg* cfg, mt_host_optimizer** out) {
+  if (!out || !store) return fail(MT_ERR_INVALID_ARG, "NULL argument");
+  *out = nullptr;
+  MT_TRY(adamw_check(cfg));
+  if (!store->master) return fail(MT_ERR_INVALID_ARG, "the optimizer needs the store's fp32 master copy");
+  auto* o = new mt_host_optimizer();
+  o->store = store;
+  o->cfg = *cfg;
+  const uint64_t n = store->G.off.record_elems * static_cast<uint64_t>(store->L);
+  o->m = static_cast<float*>(std::calloc(n, sizeof(float)));
+  o->v = static_cast<float*>(std::calloc(n, sizeof(float)));
+  if (!o->m || !o->v) {
+    mt_host_optimizer_destroy(o);
+    return fail(MT_ERR_OOM, "optimizer state allocation (%llu floats x 2) failed", (unsigned long long)n);
+  }
+  o->steps.assign(store->L, 0);
+  *out = o;
+  return MT_OK;
+}
+
+int32_t mt_host_optimizer_sink(int32_t layer, const float* host_slab, uint64_t n_elems, void* user) {
+  auto* o = static_cast<mt_host_optimizer*>(user);
+  if (!o || !host_slab || layer < 0 || layer >= o->store->L || n_elems != o->store->G.off.record_elems) return 1;
+  const mt_param_offsets& off = o->store->G.off;
+  const Geom& G = o->store->G;
+  const uint64_t base = static_cast<uint64_t>(layer) * off.record_elems;
+  float* w = o->store->master + base;
+  float* m = o->m + base;
+  float* v = o->v + base;
+  uint16_t* wb = o->store->bf + base;
+  const int64_t t = ++o->steps[layer];
+  const double bc1 = 1.0 - std::pow(static_cast<double>(o->cfg.beta1), static_cast<double>(t));
+  const double bc2 = 1.0 - std::pow(static_cast<double>(o->cfg.beta2), static_cast<double>(t));
+  // the record's tensors (its padding carries no parameter)
+  const int64_t blocks[7][2] = {
+      {static_cast<int64_t>(off.g1), G.H},
+      {static_cast<int64_t>(off.wq), G.Nqkv * G.H},
+      {static_cast<int64_t>(off.bq), G.bias ? G.Nqkv : 0},
+      {static_cast<int64_t>(off.wo), G.H * G.Nq},
+      {static_cast<int64_t>(off.g2), G.H},
+      {static_cast<int64_t>(off.wg), 2 * G.F * G.H},
+      {static_cast<int64_t>(off.wd), G.H * G.F},
+  };
+  const mt_adamw_cfg c = o->cfg;
+  const int threads = c.n_threads > 0 ? c.n_threads : default_threads();
+  for (const auto& blk : blocks) {
+    const int64_t s0 = blk[0], len = blk[1];
+    if (len == 0) continue;
+    parallel_for(len, threads, [&](int64_t a, int64_t b) {
+      adamw_range(w + s0, m + s0, v + s0, host_slab + s0, a, b, c, bc1, bc2);
+      for (int64_t i = a; i < b; ++i) {  // refresh the streamed bf16 copy (round to nearest even)
+        uint32_t u;
+        std::memcpy(&u, w + s0 + i, 4);
+        wb[s0 + i] = ((u & 0x7FFFFFFFu) > 0x7F800000u) ? static_cast<uint16_t>((u >> 16) | 0x40u)
+                                                       : static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+      }
+    });
+  }
+  return 0;
+}
+
+void mt_host_optimizer_destroy(mt_host_optimizer* o) {
+  if (!o) return;
+  std::free(o->m);
+  std::free(o->v);
+  delete o;
 }
 
 }  // extern "C"

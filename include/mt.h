@@ -324,6 +324,34 @@ mt_status mt_engine_stats(const mt_engine* e, mt_stats* out);
 mt_status mt_engine_reset(mt_engine* e);
 void mt_engine_destroy(mt_engine* e);
 
+/* ------------------------------------------------------------------------ */
+/* CPU optimizer (blog summary, design point 1: the optimizer step runs on   */
+/* the CPU with Adam momentum and variance in host memory)                   */
+/* ------------------------------------------------------------------------ */
+
+typedef struct mt_adamw_cfg {
+  float lr, beta1, beta2, eps, weight_decay;  /* AdamW, decoupled weight decay */
+  int32_t n_threads;                           /* host threads (0 = all cores, up to 32) */
+} mt_adamw_cfg;
+
+/* One AdamW step (t >= 1) on n host fp32 elements, in place:
+ * m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+ * w -= lr * (m/(1-b1^t) / (sqrt(v/(1-b2^t)) + eps) + weight_decay * w). No CUDA. */
+mt_status mt_adamw_update(float* w, float* m, float* v, const float* g, uint64_t n, const mt_adamw_cfg* cfg,
+                          int64_t t);
+
+typedef struct mt_host_optimizer mt_host_optimizer;
+
+/* AdamW state (m, v zeroed, one step counter per layer) for every record of a
+ * store that keeps its fp32 master copy. */
+mt_status mt_host_optimizer_create(mt_host_store* store, const mt_adamw_cfg* cfg, mt_host_optimizer** out);
+/* A gradient sink for mt_stream_step (user = the optimizer): applies one AdamW
+ * step to layer `layer`'s fp32 master from the gradient record and refreshes
+ * that layer's bf16 streaming copy (round to nearest even). Returns 0, or 1 on
+ * a mismatched layer or record size. */
+int32_t mt_host_optimizer_sink(int32_t layer, const float* host_slab, uint64_t n_elems, void* user);
+void mt_host_optimizer_destroy(mt_host_optimizer* o);
+
 /* Host-side schedule (no CUDA): for n_layers and interval K, the sequence of
  * layer uses in compute order and, for a pool of n_slots weight buffers, the
  * slot of each use and whether it needs a fresh copy (furthest-next-use

@@ -29,3 +29,4 @@ from .layer import (  # noqa: F401
     swiglu_bwd,
     swiglu_fwd,
 )
+from .optimizer import adamw_step  # noqa: F401

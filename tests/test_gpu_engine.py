@@ -196,3 +196,47 @@ def test_slow_sink_times_out_with_a_clean_status():
         assert sorted(g) == [0, 1, 2]
     finally:
         s.close()
+
+
+def test_cpu_optimizer_sink_closes_the_training_loop():
+    """The library's AdamW sink updates each layer's fp32 master from its streamed
+    gradient record and refreshes the bf16 copy the next step streams."""
+    from oracle.optimizer import adamw_step
+    ref = Stack(TINY, 3, 2, 128, ckpt_interval=2)
+    try:
+        _, _, grads = ref.step()
+    finally:
+        ref.close()
+    s = Stack(TINY, 3, 2, 128, ckpt_interval=2)
+    cfg = L.mt_adamw_cfg(1e-2, 0.9, 0.95, 1e-8, 0.1, 0)
+    opt = L.mt_host_optimizer_create(s.store, cfg)
+    try:
+        off = L.mt_layer_param_offsets(s.cfg)
+        n = off.record_elems
+        masters0 = [np.ctypeslib.as_array((ctypes.c_float * n).from_address(L.mt_host_store_master(s.store, l))).copy()
+                    for l in range(3)]
+        import torch
+        x_d, dy_d = H.dev_bf16(s.x), H.dev_bf16(s.dy)
+        y = H.empty_bf16(2, 128, TINY["hidden"])
+        dx = H.empty_bf16(2, 128, TINY["hidden"])
+        L.mt_stream_step(s.eng, s.store, x_d, dy_d, y, dx, L.optimizer_sink(), opt)
+        torch.cuda.synchronize()
+        for l in range(3):
+            master = np.ctypeslib.as_array((ctypes.c_float * n).from_address(L.mt_host_store_master(s.store, l)))
+            bf = np.ctypeslib.as_array((ctypes.c_uint16 * n).from_address(L.mt_host_store_bf16(s.store, l)))
+            g = grads[l].astype(np.float64)
+            used = np.zeros(n, dtype=bool)
+            for name, shp in synth.layer_tensor_shapes(**H.shape_dict(s.cfg)).items():
+                o = getattr(off, name)
+                used[o:o + int(np.prod(shp))] = True
+            w_ref, _, _ = adamw_step(masters0[l][used], 0.0, 0.0, g[used], 1, 1e-2, 0.9, 0.95, 1e-8, 0.1)
+            assert np.max(np.abs(master[used] - w_ref)) < 1e-5
+            assert np.array_equal(bf[used], synth.f32_to_bf16_bits(master[used]))
+        # the next step streams the updated weights
+        y2 = H.empty_bf16(2, 128, TINY["hidden"])
+        L.mt_stream_step(s.eng, s.store, x_d, dy_d, y2, dx, L.optimizer_sink(), opt)
+        torch.cuda.synchronize()
+        assert not torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    finally:
+        L.mt_host_optimizer_destroy(opt)
+        s.close()

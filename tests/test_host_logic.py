@@ -136,3 +136,24 @@ def test_tflops_formula_reproduces_table7_long_context_rows():
         tf = metrics.sustained_tflops(m["N"], m["L"], m["H"], r["B"], r["T"], r["step_s"])
         assert abs(tf - r["tflops"]) / r["tflops"] < 1e-3, (r, tf)
     assert metrics.tokens_per_s(96, 1024, 2.0) == 49152.0
+
+
+def test_cpu_adamw_matches_oracle_over_three_steps():
+    import numpy as np
+
+    from oracle.optimizer import adamw_step
+    rng = np.random.default_rng(61)
+    n = 3_000_001  # several threads' worth, odd length
+    w = rng.standard_normal(n).astype(np.float32)
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    cfg = L.mt_adamw_cfg(1e-3, 0.9, 0.95, 1e-8, 0.01, 0)
+    w64, m64, v64 = w.astype(np.float64), m.astype(np.float64), v.astype(np.float64)
+    for t in range(1, 4):
+        g = rng.standard_normal(n).astype(np.float32)
+        L.mt_adamw_update(w, m, v, g, n, cfg, t)
+        w64, m64, v64 = adamw_step(w64, m64, v64, g.astype(np.float64), t, 1e-3, 0.9, 0.95, 1e-8, 0.01)
+    assert np.max(np.abs(w - w64)) < 1e-6
+    assert np.max(np.abs(m - m64)) < 1e-6 and np.max(np.abs(v - v64)) < 1e-6
+    with pytest.raises(L.MTError):
+        L.mt_adamw_update(w, m, v, g, n, cfg, 0)

@@ -315,3 +315,34 @@ def test_weight_gradient_against_textbook_loops():
         for f in range(F):
             s = sum(dy[b, t, i] * m[b, t, f] for b in range(2) for t in range(3))
             assert abs(gr["wd"][i, f] - s) < 1e-12
+
+
+# ------------------------------------------------------------ AdamW
+from oracle.optimizer import adamw_step  # noqa: E402
+
+
+def test_adamw_first_step_closed_form():
+    rng = np.random.default_rng(51)
+    w = rng.standard_normal(50)
+    g = rng.standard_normal(50)
+    lr, eps, wd = 1e-3, 1e-8, 0.1
+    w1, m1, v1 = adamw_step(w, np.zeros(50), np.zeros(50), g, 1, lr, 0.9, 0.999, eps, wd)
+    np.testing.assert_allclose(m1, 0.1 * g, rtol=1e-12)
+    np.testing.assert_allclose(v1, 0.001 * g * g, rtol=1e-12)
+    # bias correction makes the first step lr * g / (|g| + eps) plus the decoupled decay
+    np.testing.assert_allclose(w1, w - lr * (g / (np.abs(g) + eps) + wd * w), rtol=1e-12, atol=1e-15)
+
+
+def test_adamw_zero_gradient_only_decays():
+    w = np.linspace(-2, 2, 9)
+    w1, m1, v1 = adamw_step(w, np.zeros(9), np.zeros(9), np.zeros(9), 1, 0.01, 0.9, 0.999, 1e-8, 0.5)
+    np.testing.assert_array_equal(m1, 0.0)
+    np.testing.assert_allclose(w1, w * (1 - 0.01 * 0.5), rtol=1e-15)
+
+
+def test_adamw_constant_gradient_moves_by_lr_per_step():
+    g = np.array([3.0, -0.5, 1e-3])
+    w, m, v = np.zeros(3), np.zeros(3), np.zeros(3)
+    for t in range(1, 6):
+        w, m, v = adamw_step(w, m, v, g, t, 0.01, 0.9, 0.99, 1e-12, 0.0)
+    np.testing.assert_allclose(w, -5 * 0.01 * g / (np.abs(g) + 1e-12), rtol=1e-9)

@@ -71,6 +71,27 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def gemm_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, when that summary
+    was taken on this workload with the current GEMM source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "gemm2_kernel_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    csrc = os.path.join(ROOT, "host_offloaded_layer_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "tcgen05.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    if kv.get("kernel_source_sha256") != h.hexdigest() or kv.get("workload") != workload:
+        return None
+    return float(kv["dram_bytes_per_launch"])
+
+
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
@@ -350,9 +371,10 @@ def run_ours(args, cfg, rank, world, local_rank):
             "e2e": {"value": e2e, "unit": UNIT,
                     "h2d_bytes_per_step": int(st_e2e.h2d_bytes), "d2h_bytes_per_step": int(st_e2e.d2h_bytes)},
             "gpu_launches": int(st.kernel_launches) * args.steps,
-            "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05)", "achieved": gemm_tf,
+            "roofline": {"bound": "tensor", "kernel": "gemm2_kernel (tcgen05, 2-SM)", "achieved": gemm_tf,
                          "peak": peak_tf, "unit": "TFLOP/s", "frac": (gemm_tf / peak_tf) if gemm_tf else None,
-                         "traffic": None, "peak_source": f"{src} bf16_tflops_sustained",
+                         "traffic": gemm_traffic(cfg["name"]), "traffic_unit": "bytes per launch",
+                         "peak_source": f"{src} bf16_tflops_sustained",
                          "gemm_launches_per_step": int(st.gemm_launches)},
             "step_roofline": {"t_roof_ms": t_roof * 1e3, "t_step_ms": ms, "frac": t_roof / (ms / 1e3),
                               "t_compute_ms": t_comp * 1e3, "t_h2d_ms": t_h2d * 1e3, "t_d2h_ms": t_d2h * 1e3,

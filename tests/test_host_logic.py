@@ -157,3 +157,18 @@ def test_cpu_adamw_matches_oracle_over_three_steps():
     assert np.max(np.abs(m - m64)) < 1e-6 and np.max(np.abs(v - v64)) < 1e-6
     with pytest.raises(L.MTError):
         L.mt_adamw_update(w, m, v, g, n, cfg, 0)
+
+
+def test_bench_reference_arm_prints_one_json_line():
+    """`bench.py --impl reference` times the CPU oracle and prints the contract's line."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "1",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOPS" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0

@@ -110,8 +110,6 @@ _SIGS = {
     "mt_schedule": (c_i32, [c_i32, c_i32, c_i32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32),
                             ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
 }
-_STATUS_FUNCS = {n for n, (r, _) in _SIGS.items() if r is c_i32 and n not in ("mt_schedule_len",)}
-
 _lib: ctypes.CDLL | None = None
 
 

@@ -33,22 +33,36 @@ constexpr int ATOM = 128 * 64 * 2;  // 16 KiB
 // shared memory: Q | K0 V0 | K1 V1 | P0 | P1
 constexpr int OFF_Q = 0, OFF_KV = TILE, OFF_P = 5 * TILE;
 constexpr int SMEM_TILES = 7 * TILE;
-constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;
-constexpr int NUM_THREADS = 192;
+constexpr int SMEM_BYTES = SMEM_TILES + 128 + 1024 + 1024;  // tiles, barriers, row exchange, alignment
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_O = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
+// Bounded barrier among a group of threads built on an mbarrier initialised
+// with the group's size: arrive, then wait (bounded) for the phase to flip.
+// `phase` counts this thread's uses. Returns false when the wait ran out.
+__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag, int32_t* err) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE);
+  ++phase;
+  return ok;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// NG softmax warpgroups: with NG = 2, warps 2-5 take key columns 0-63 (and O
+// columns 0-63) of the 128 rows, warps 6-9 columns 64-127 of the same rows;
+// the two halves of each row maximum and row sum meet in shared memory.
+template <int NG>
+__global__ void __launch_bounds__(64 + 128 * NG, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16* __restrict__ o, int64_t ld_o,
                        float* __restrict__ lse, int T, int nq, int nkv, float scale_log2, int32_t* err) {
+  constexpr int SCOLS = BKV / NG, OCOLS = D / NG;  // S and O columns per softmax group
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
@@ -58,8 +72,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* s_full = bars + 5;      // 2
   uint64_t* p_full = bars + 7;      // 2
   uint64_t* o_done = bars + 9;      // 2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* x_bar = bars + 11;      // 1: row exchange between the softmax groups
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xch = reinterpret_cast<float*>(smem + SMEM_TILES + 128);  // [NG][128] row halves
 
   const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -76,9 +92,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&kv_full[i]), 1);
       mbar_init(smem_u32(&kv_empty[i]), 1);
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), 128);
+      mbar_init(smem_u32(&p_full[i]), 128 * NG);
       mbar_init(smem_u32(&o_done[i]), 1);
     }
+    mbar_init(smem_u32(x_bar), 128 * NG);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
@@ -163,12 +180,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
     }
   } else {
-    // ------------------------------------------------------------ softmax (one thread per query row)
-    const int qw = warp & 3;  // TMEM lanes [32 qw, 32 qw + 32)
+    // ------------------------------------------------------------ softmax (one thread per query row and group)
+    const int g = (warp - 2) >> 2;  // softmax group: columns [g*SCOLS, (g+1)*SCOLS) of S
+    const int qw = warp & 3;        // TMEM lanes [32 qw, 32 qw + 32)
     const int r = qw * 32 + lane;
     const int q_row = q0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
+    uint32_t xph = 0;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
@@ -177,25 +196,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       fence_after();
-      float sv[BKV];
+      float sv[SCOLS];
 #pragma unroll
-      for (int ch = 0; ch < BKV / 32; ++ch) {
+      for (int ch = 0; ch < SCOLS / 32; ++ch) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + COL_S0 + s * BKV + ch * 32, u);
+        tmem_ld32(tmem + lane_base + COL_S0 + s * BKV + g * SCOLS + ch * 32, u);
 #pragma unroll
         for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
       }
-      const int k0 = j * BKV;
-      const bool diag = k0 + BKV - 1 > q0;
+      const int k0 = j * BKV + g * SCOLS;
+      const bool diag = k0 + SCOLS - 1 > q0;
       float mx = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < BKV; ++e) {
+      for (int e = 0; e < SCOLS; ++e) {
         float v = sv[e] * scale_log2;
         if (diag && k0 + e > q_row) v = -INFINITY;
         sv[e] = v;
         mx = fmaxf(mx, v);
       }
+      if (NG == 2) {  // the other half of the row's maximum
+        xch[g * 128 + r] = mx;
+        if (!group_sync(smem_u32(x_bar), xph, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, xch[(g ^ 1) * 128 + r]);
+        if (!group_sync(smem_u32(x_bar), xph, abort_flag, err)) {  // both halves read before the next write
+          ok = false;
+          break;
+        }
+      }
       // rescale O only when some row of the warp raised its maximum by more than the threshold
+      // (the decision is the same in both groups: it depends on the row maximum only)
       const bool need = (m_run == -INFINITY) || (mx > m_run + RESCALE_THRESHOLD);
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = fmaxf(m_run, mx);
@@ -209,12 +241,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           fence_after();
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
+          for (int ch = 0; ch < OCOLS / 32; ++ch) {
             uint32_t u[32];
-            tmem_ld32(tmem + lane_base + COL_O + ch * 32, u);
+            const uint32_t col = COL_O + g * OCOLS + ch * 32;
+            tmem_ld32(tmem + lane_base + col, u);
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(tmem + lane_base + COL_O + ch * 32, u);
+            tmem_st32(tmem + lane_base + col, u);
           }
         }
         l_run *= alpha;
@@ -230,7 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint8_t* prow = smem + OFF_P + s * TILE + r * 128;
       float lsum = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < BKV / 8; ++ch) {  // 16-byte chunks of 8 columns
+      for (int ch = 0; ch < SCOLS / 8; ++ch) {  // 16-byte chunks of 8 columns
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -242,7 +275,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         w.y = pack_bf16(p[2], p[3]);
         w.z = pack_bf16(p[4], p[5]);
         w.w = pack_bf16(p[6], p[7]);
-        const int atom = ch >> 3, c16 = ch & 7;
+        const int cg = g * (SCOLS / 8) + ch;  // chunk index within the row of 128 columns
+        const int atom = cg >> 3, c16 = cg & 7;
         *reinterpret_cast<uint4*>(prow + atom * ATOM + ((c16 ^ (r & 7)) << 4)) = w;
       }
       l_run += lsum;
@@ -250,16 +284,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_before();
       mbar_arrive(smem_u32(&p_full[s]));
     }
+    float l_tot = l_run;
+    if (NG == 2 && ok) {
+      xch[g * 128 + r] = l_run;
+      ok = group_sync(smem_u32(x_bar), xph, abort_flag, err);
+      l_tot = l_run + xch[(g ^ 1) * 128 + r];
+    }
     if (ok && n_kv > 0) {
       const int jl = n_kv - 1;
       if (warp_wait(smem_u32(&o_done[jl & 1]), (jl >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
         fence_after();
-        const float inv = 1.f / l_run;
+        const float inv = 1.f / l_tot;
         __nv_bfloat16* orow = o + (static_cast<int64_t>(row0) + q_row) * ld_o + static_cast<int64_t>(h) * D;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < OCOLS / 32; ++ch) {
           uint32_t u[32];
-          tmem_ld32(tmem + lane_base + COL_O + ch * 32, u);
+          const int oc = g * OCOLS + ch * 32;
+          tmem_ld32(tmem + lane_base + COL_O + oc, u);
           if (q_row < T) {
 #pragma unroll
             for (int qd = 0; qd < 4; ++qd) {
@@ -268,11 +309,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               w.y = pack_bf16(__uint_as_float(u[qd * 8 + 2]) * inv, __uint_as_float(u[qd * 8 + 3]) * inv);
               w.z = pack_bf16(__uint_as_float(u[qd * 8 + 4]) * inv, __uint_as_float(u[qd * 8 + 5]) * inv);
               w.w = pack_bf16(__uint_as_float(u[qd * 8 + 6]) * inv, __uint_as_float(u[qd * 8 + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + ch * 32 + qd * 8) = w;
+              *reinterpret_cast<uint4*>(orow + oc + qd * 8) = w;
             }
           }
         }
-        if (q_row < T) lse[(static_cast<int64_t>(b) * nq + h) * T + q_row] = (m_run + log2f(l_run)) * LN2;
+        if (q_row < T && g == 0) lse[(static_cast<int64_t>(b) * nq + h) * T + q_row] = (m_run + log2f(l_tot)) * LN2;
       }
     }
   }
@@ -291,10 +332,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ld_qkv a multiple of 8 (checked by the caller).
 mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T,
                              int nq, int nkv, cudaStream_t st) {
+  constexpr int NG = 2;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    attr = cudaFuncSetAttribute(attn_fwd_tc_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr != cudaSuccess) return fail(MT_ERR_CUDA, "attention smem attribute: %s", cudaGetErrorString(attr));
   CUtensorMap tm;
@@ -304,8 +346,8 @@ mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
   dim3 grid((T + BQ - 1) / BQ, nq, B);
   const float scale_log2 = LOG2E / sqrtf(static_cast<float>(D));
-  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, lse, T, nq,
-                                                            nkv, scale_log2, err);
+  attn_fwd_tc_kernel<NG><<<grid, 64 + 128 * NG, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, lse,
+                                                                  T, nq, nkv, scale_log2, err);
   MT_TRY(launch_check("attn_fwd_tc_kernel"));
   add_exec_flops(4.0 * B * nq * D * (0.5 * double(T) * double(T)));
   return MT_OK;
@@ -335,12 +377,11 @@ constexpr int KV_OFF_LD = KV_OFF_PD + 4 * ATOM;
 constexpr int KV_SMEM_TILES = KV_OFF_LD + 4 * 64 * 4;
 constexpr int KV_SMEM_BYTES = KV_SMEM_TILES + 256 + 1024;
 constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;
+// Both backward kernels run two groups of four compute warps (warps 2-5 and 6-9),
+// each on half of a block's 64 columns: no row reduction crosses the halves.
+constexpr int BWD_THREADS = 64 + 256;
 
-__device__ __forceinline__ void named_sync_compute() {  // the 128 threads of warps 2-5
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
                            const __grid_constant__ CUtensorMap tm_do64, const float* __restrict__ lse,
                            const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int T,
@@ -356,7 +397,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* pd_full = bars + 7;   // 2
   uint64_t* mma_done = bars + 9;  // 2
   uint64_t* fin = bars + 11;      // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* l_bar = bars + 12;    // 1: lse/delta of a block written by the 128 compute threads
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int kb = blockIdx.x;  // small key blocks have the most query blocks: first
@@ -378,9 +420,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&qo_full[i]), 1);
       mbar_init(smem_u32(&qo_empty[i]), 1);
       mbar_init(smem_u32(&sp_full[i]), 1);
-      mbar_init(smem_u32(&pd_full[i]), 128);
+      mbar_init(smem_u32(&pd_full[i]), 256);
       mbar_init(smem_u32(&mma_done[i]), 1);
     }
+    mbar_init(smem_u32(l_bar), 256);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -483,49 +526,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) umma_commit(smem_u32(fin));
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ P^T / dS^T, one thread per key row
+    // ------------------------------------------------------------ P^T / dS^T, one thread per key row and group
+    const int g = (warp - 2) >> 2;  // query columns [32 g, 32 g + 32) of each 64-column block
     const int qw = warp & 3;
     const int r = qw * 32 + lane;  // key row within the block
-    const int t = threadIdx.x - 64;  // 0..127 among the compute threads
+    const int t = threadIdx.x - 64;  // 0..255 among the compute threads
     const int kv_row = k0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
+    uint32_t lph = 0;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
       const int h = c * grp + it / per_head;
       const int q0 = (qb0 + it % per_head) * 64;
       {  // this block's log-sum-exp (log2 domain) and delta, shared by all key rows
-        const int q = q0 + (t & 63);
-        const int64_t sb = (static_cast<int64_t>(b) * nq + h) * T;
-        if (t < 64)
-          lsd[st * 128 + t] = q < T ? lse[sb + q] * LOG2E : INFINITY;
-        else
-          lsd[st * 128 + t] = q < T ? delta[sb + q] : 0.f;
-        named_sync_compute();
+        if (t < 128) {
+          const int q = q0 + (t & 63);
+          const int64_t sb = (static_cast<int64_t>(b) * nq + h) * T;
+          if (t < 64)
+            lsd[st * 128 + t] = q < T ? lse[sb + q] * LOG2E : INFINITY;
+          else
+            lsd[st * 128 + t] = q < T ? delta[sb + q] : 0.f;
+        }
+        if (!group_sync(smem_u32(l_bar), lph, abort_flag, err)) {
+          ok = false;
+          break;
+        }
       }
       if (!warp_wait(smem_u32(&sp_full[st]), (it >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
         ok = false;
         break;
       }
       fence_after();
-      float sv[64], dv[64];
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      float sv[32], dv[32];
+      {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + KV_COL_ST + st * 64 + ch * 32, u);
+        tmem_ld32(tmem + lane_base + KV_COL_ST + st * 64 + g * 32, u);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
-        tmem_ld32(tmem + lane_base + KV_COL_DPT + st * 64 + ch * 32, u);
+        for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
+        tmem_ld32(tmem + lane_base + KV_COL_DPT + st * 64 + g * 32, u);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dv[ch * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
       }
-      const float* L2 = lsd + st * 128;
+      const float* L2 = lsd + st * 128 + g * 32;
       const float* Dl = L2 + 64;
-      const bool diag = q0 < k0 + 127;
+      const int qc0 = q0 + g * 32;
+      const bool diag = qc0 < k0 + 127;
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
+      for (int e = 0; e < 32; ++e) {
         float p = exp2f(sv[e] * scale_log2 - L2[e]);
-        if (diag && kv_row > q0 + e) p = 0.f;
+        if (diag && kv_row > qc0 + e) p = 0.f;
         sv[e] = p;
         dv[e] = p * (dv[e] - Dl[e]);
       }
@@ -537,16 +587,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       uint8_t* prow = smem + KV_OFF_PD + st * 2 * ATOM + r * 128;
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c16 = g * 4 + ch;
         uint4 wp, wd;
-        wp.x = pack_bf16(sv[c16 * 8 + 0], sv[c16 * 8 + 1]);
-        wp.y = pack_bf16(sv[c16 * 8 + 2], sv[c16 * 8 + 3]);
-        wp.z = pack_bf16(sv[c16 * 8 + 4], sv[c16 * 8 + 5]);
-        wp.w = pack_bf16(sv[c16 * 8 + 6], sv[c16 * 8 + 7]);
-        wd.x = pack_bf16(dv[c16 * 8 + 0], dv[c16 * 8 + 1]);
-        wd.y = pack_bf16(dv[c16 * 8 + 2], dv[c16 * 8 + 3]);
-        wd.z = pack_bf16(dv[c16 * 8 + 4], dv[c16 * 8 + 5]);
-        wd.w = pack_bf16(dv[c16 * 8 + 6], dv[c16 * 8 + 7]);
+        wp.x = pack_bf16(sv[ch * 8 + 0], sv[ch * 8 + 1]);
+        wp.y = pack_bf16(sv[ch * 8 + 2], sv[ch * 8 + 3]);
+        wp.z = pack_bf16(sv[ch * 8 + 4], sv[ch * 8 + 5]);
+        wp.w = pack_bf16(sv[ch * 8 + 6], sv[ch * 8 + 7]);
+        wd.x = pack_bf16(dv[ch * 8 + 0], dv[ch * 8 + 1]);
+        wd.y = pack_bf16(dv[ch * 8 + 2], dv[ch * 8 + 3]);
+        wd.z = pack_bf16(dv[ch * 8 + 4], dv[ch * 8 + 5]);
+        wd.w = pack_bf16(dv[ch * 8 + 6], dv[ch * 8 + 7]);
         const int sw = (c16 ^ (r & 7)) << 4;
         *reinterpret_cast<uint4*>(prow + sw) = wp;
         *reinterpret_cast<uint4*>(prow + ATOM + sw) = wd;
@@ -558,8 +609,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok && n_it > 0 && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
       fence_after();
       __nv_bfloat16* drow = dqkv + (static_cast<int64_t>(row0) + kv_row) * ld;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {  // 0: dK (scaled), 1: dV
+      {
+        const int which = g;  // group 0 writes dK (scaled), group 1 dV
         const uint32_t col = which == 0 ? KV_COL_DK : KV_COL_DV;
         const float f = which == 0 ? scale : 1.f;
         __nv_bfloat16* out = drow + (which == 0 ? col_k : col_v);
@@ -598,7 +649,7 @@ constexpr int DQ_SMEM_TILES = DQ_OFF_DS + 2 * ATOM;
 constexpr int DQ_SMEM_BYTES = DQ_SMEM_TILES + 256 + 1024;
 constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
                           const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
                           const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int T, int nq,
@@ -632,7 +683,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&kv_full[i]), 1);
       mbar_init(smem_u32(&kv_empty[i]), 1);
       mbar_init(smem_u32(&sp_full[i]), 1);
-      mbar_init(smem_u32(&ds_full[i]), 128);
+      mbar_init(smem_u32(&ds_full[i]), 256);
       mbar_init(smem_u32(&mma_done[i]), 1);
     }
     *abort_flag = 0;
@@ -728,6 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) umma_commit(smem_u32(fin));
     __syncwarp();
   } else {
+    const int g = (warp - 2) >> 2;  // key columns [32 g, 32 g + 32) of each 64-column block
     const int qw = warp & 3;
     const int r = qw * 32 + lane;
     const int q_row = q0 + r;
@@ -743,21 +795,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       fence_after();
-      float sv[64], dv[64];
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      float sv[32], dv[32];
+      {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + DQ_COL_S + st * 64 + ch * 32, u);
+        tmem_ld32(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, u);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
-        tmem_ld32(tmem + lane_base + DQ_COL_DP + st * 64 + ch * 32, u);
+        for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
+        tmem_ld32(tmem + lane_base + DQ_COL_DP + st * 64 + g * 32, u);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dv[ch * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
       }
-      const int k0 = j * 64;
-      const bool diag = k0 + 63 > q0;
+      const int k0 = j * 64 + g * 32;
+      const bool diag = k0 + 31 > q0;
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
+      for (int e = 0; e < 32; ++e) {
         float p = exp2f(sv[e] * scale_log2 - lse2);
         if (diag && k0 + e > q_row) p = 0.f;
         dv[e] = p * (dv[e] - dl);
@@ -770,12 +821,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       uint8_t* drow = smem + DQ_OFF_DS + st * ATOM + r * 128;
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c16 = g * 4 + ch;
         uint4 w;
-        w.x = pack_bf16(dv[c16 * 8 + 0], dv[c16 * 8 + 1]);
-        w.y = pack_bf16(dv[c16 * 8 + 2], dv[c16 * 8 + 3]);
-        w.z = pack_bf16(dv[c16 * 8 + 4], dv[c16 * 8 + 5]);
-        w.w = pack_bf16(dv[c16 * 8 + 6], dv[c16 * 8 + 7]);
+        w.x = pack_bf16(dv[ch * 8 + 0], dv[ch * 8 + 1]);
+        w.y = pack_bf16(dv[ch * 8 + 2], dv[ch * 8 + 3]);
+        w.z = pack_bf16(dv[ch * 8 + 4], dv[ch * 8 + 5]);
+        w.w = pack_bf16(dv[ch * 8 + 6], dv[ch * 8 + 7]);
         *reinterpret_cast<uint4*>(drow + ((c16 ^ (r & 7)) << 4)) = w;
       }
       fence_proxy_async_smem();
@@ -784,11 +836,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if (ok && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
       fence_after();
-      __nv_bfloat16* out = dqkv + (static_cast<int64_t>(row0) + q_row) * ld + static_cast<int64_t>(h) * D;
+      __nv_bfloat16* out = dqkv + (static_cast<int64_t>(row0) + q_row) * ld + static_cast<int64_t>(h) * D + g * 64;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {  // group g writes dQ columns [64 g, 64 g + 64)
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + DQ_COL_DQ + ch * 32, u);
+        tmem_ld32(tmem + lane_base + DQ_COL_DQ + g * 64 + ch * 32, u);
         if (q_row < T) {
 #pragma unroll
           for (int qd = 0; qd < 4; ++qd) {
@@ -838,11 +890,11 @@ mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o,
   const float scale_log2 = LOG2E * scale;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(dqkv);
   dim3 gq((T + 127) / 128, nq, B);
-  attn_bwd_dq_tc_kernel<<<gq, NUM_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, T, nq, nkv,
+  attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, T, nq, nkv,
                                                                 scale_log2, scale, err);
   MT_TRY(launch_check("attn_bwd_dq_tc_kernel"));
   dim3 gk((T + 127) / 128, nkv, B);
-  attn_bwd_dkv_tc_kernel<<<gk, NUM_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, T, nq, nkv,
+  attn_bwd_dkv_tc_kernel<<<gk, BWD_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, T, nq, nkv,
                                                                  scale_log2, scale, err);
   MT_TRY(launch_check("attn_bwd_dkv_tc_kernel"));
   // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)

@@ -307,14 +307,16 @@ void sink_loop(mt_engine* e, mt_grad_sink sink, void* user) {
     }
     const auto deadline = Clock::now() + std::chrono::milliseconds(e->opts.timeout_ms);
     mt_status s = poll_event(e->d2h_done[it.jb], deadline, "gradient offload");
+    double sink_ms = 0.0;
     if (s == MT_OK && sink) {
       const auto t0 = Clock::now();
       int32_t rc = sink(it.layer, it.ptr, rec, user);
-      e->st.sink_ms += std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
+      sink_ms = std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
       if (rc != 0) s = fail(MT_ERR_SINK, "gradient sink returned %d for layer %d", rc, it.layer);
     }
     if (it.slab < 0) cudaFreeHost(it.ptr);  // no pool: the record was pinned for this layer only
     std::lock_guard<std::mutex> lk(e->mu);
+    e->st.sink_ms += sink_ms;
     if (it.slab >= 0) e->free_slabs.push_back(it.slab);
     if (s != MT_OK) {
       e->sink_status = s;
@@ -619,7 +621,10 @@ mt_status mt_stream_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, 
   const double f0 = exec_flops_counter();
   const uint64_t k0 = launch_counter();
   const uint64_t h2d0 = e->st.h2d_bytes, d2h0 = e->st.d2h_bytes;
-  e->st.sink_ms = 0;
+  {
+    std::lock_guard<std::mutex> lk(e->mu);
+    e->st.sink_ms = 0;
+  }
   e->timer.n = 0;
   e->timer.flops.clear();
   e->timer.overflow = false;

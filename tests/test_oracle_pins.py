@@ -346,3 +346,55 @@ def test_adamw_constant_gradient_moves_by_lr_per_step():
     for t in range(1, 6):
         w, m, v = adamw_step(w, m, v, g, t, 0.01, 0.9, 0.99, 1e-12, 0.0)
     np.testing.assert_allclose(w, -5 * 0.01 * g / (np.abs(g) + 1e-12), rtol=1e-9)
+
+
+# ------------------------------------------------------------ embedding, LM head, cross-entropy
+from oracle import head as HD  # noqa: E402
+
+
+def test_head_loss_gradients_match_central_differences():
+    rng = np.random.default_rng(71)
+    B, T, H, V = 2, 3, 8, 11
+    y = rng.standard_normal((B, T, H))
+    gf = 1.0 + 0.2 * rng.standard_normal(H)
+    W = 0.5 * rng.standard_normal((V, H))
+    tgt = rng.integers(0, V, size=(B, T))
+    loss, dy, dgf, dW = HD.head_loss_fwd_bwd(y, gf, W, tgt, 1e-6)
+    h = 1e-6
+    for arr, g, name in ((y, dy, "y"), (gf, dgf, "gf"), (W, dW, "W")):
+        e = rng.standard_normal(arr.shape)
+        args_p = {"y": y, "gf": gf, "W": W}
+        args_m = dict(args_p)
+        args_p[name] = arr + h * e
+        args_m[name] = arr - h * e
+        lp = HD.head_loss_fwd_bwd(args_p["y"], args_p["gf"], args_p["W"], tgt, 1e-6)[0]
+        lm = HD.head_loss_fwd_bwd(args_m["y"], args_m["gf"], args_m["W"], tgt, 1e-6)[0]
+        assert abs((lp - lm) / (2 * h) - np.sum(g * e)) < 1e-7, name
+
+
+def test_head_loss_closed_forms():
+    # all-zero logits: every token's loss is log V, and each dW row is the softmax-minus-onehot weighting
+    B, T, H, V = 1, 4, 6, 5
+    y = np.random.default_rng(72).standard_normal((B, T, H))
+    W = np.zeros((V, H))
+    tgt = np.array([[0, 1, 1, 4]])
+    loss, dy, dgf, dW = HD.head_loss_fwd_bwd(y, np.ones(H), W, tgt, 1e-6)
+    assert abs(loss - np.log(V)) < 1e-12
+    assert np.all(dy == 0) and np.all(dgf == 0)
+    h, _ = O.rmsnorm_fwd(y, np.ones(H), 1e-6)
+    counts = np.bincount(tgt.reshape(-1), minlength=V)
+    expect = (h.reshape(-1, H).sum(axis=0)[None, :] / V - np.stack(
+        [h.reshape(-1, H)[tgt.reshape(-1) == v].sum(axis=0) for v in range(V)])) / (B * T)
+    np.testing.assert_allclose(dW, expect, atol=1e-14)
+    assert counts.sum() == B * T
+
+
+def test_embedding_backward_is_a_scatter_add():
+    rng = np.random.default_rng(73)
+    tok = np.array([[3, 1, 3], [0, 3, 2]])
+    dx = rng.standard_normal((2, 3, 4))
+    dE = HD.embed_bwd(tok, dx, 5)
+    np.testing.assert_allclose(dE[3], dx[0, 0] + dx[0, 2] + dx[1, 1], atol=1e-15)
+    np.testing.assert_array_equal(dE[4], 0.0)
+    E = rng.standard_normal((5, 4))
+    np.testing.assert_array_equal(HD.embed_fwd(tok, E)[1, 2], E[2])

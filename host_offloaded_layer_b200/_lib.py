@@ -102,6 +102,12 @@ _SIGS = {
     "mt_engine_stats": (c_i32, [c_vp, ctypes.POINTER(mt_stats)]),
     "mt_engine_reset": (c_i32, [c_vp]),
     "mt_engine_destroy": (None, [c_vp]),
+    "mt_embed_fwd": (c_i32, [_P, _P, _P, c_i64, c_i32, c_i32, _P, _P]),
+    "mt_embed_sort": (c_i32, [_P, c_i64, c_i32, _P, _P]),
+    "mt_embed_bwd": (c_i32, [_P, _P, _P, _P, c_i32, c_i32, _P]),
+    "mt_head_workspace_bytes": (c_u64, [c_i64, c_i32, c_i32, c_i32]),
+    "mt_head_loss_fwd_bwd": (c_i32, [_P, _P, _P, _P, c_i64, c_i32, c_i32, c_f32, c_i32, _P, _P, _P, _P, _P, c_u64,
+                                     _P]),
     "mt_adamw_update": (c_i32, [_P, _P, _P, _P, c_u64, ctypes.POINTER(mt_adamw_cfg), c_i64]),
     "mt_host_optimizer_create": (c_i32, [c_vp, ctypes.POINTER(mt_adamw_cfg), ctypes.POINTER(c_vp)]),
     "mt_host_optimizer_sink": (c_i32, [c_i32, ctypes.POINTER(c_f32), c_u64, c_vp]),
@@ -344,3 +350,25 @@ def mt_host_optimizer_destroy(opt):
 def optimizer_sink():
     """The library's AdamW sink as a callable for mt_stream_step (pass the optimizer as `user`)."""
     return ctypes.cast(load().mt_host_optimizer_sink, mt_grad_sink)
+
+
+def mt_embed_fwd(tokens, E, x, M, H, V, bad_tokens, stream=None):
+    _check(load().mt_embed_fwd(_ptr(tokens), _ptr(E), _ptr(x), M, H, V, _ptr(bad_tokens), _stream(stream)))
+
+
+def mt_embed_sort(tokens, M, V, order, start):
+    _check(load().mt_embed_sort(_ptr(tokens), M, V, _ptr(order), _ptr(start)))
+
+
+def mt_embed_bwd(order, start, dx, dE, H, V, stream=None):
+    _check(load().mt_embed_bwd(_ptr(order), _ptr(start), _ptr(dx), _ptr(dE), H, V, _stream(stream)))
+
+
+def mt_head_workspace_bytes(M, H, V, vocab_chunk) -> int:
+    return load().mt_head_workspace_bytes(M, H, V, vocab_chunk)
+
+
+def mt_head_loss_fwd_bwd(y, gf, W, targets, M, H, V, eps, vocab_chunk, loss, dy, dgf, dW, ws, ws_bytes, stream=None):
+    _check(load().mt_head_loss_fwd_bwd(_ptr(y), _ptr(gf), _ptr(W), _ptr(targets), M, H, V, eps, vocab_chunk,
+                                       _ptr(loss), _ptr(dy), _ptr(dgf), _ptr(dW), _ptr(ws), ws_bytes,
+                                       _stream(stream)))

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmt.so")
-SOURCES = ["common.cu", "gemm.cu", "elementwise.cu", "attention.cu", "attention_tc.cu", "layer.cu", "engine.cu"]
+SOURCES = ["common.cu", "gemm.cu", "elementwise.cu", "attention.cu", "attention_tc.cu", "layer.cu", "engine.cu", "head.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

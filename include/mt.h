@@ -325,6 +325,38 @@ mt_status mt_engine_reset(mt_engine* e);
 void mt_engine_destroy(mt_engine* e);
 
 /* ------------------------------------------------------------------------ */
+/* Embedding, final norm, LM head and loss (the pages count embedding and   */
+/* head in the parameters, Table 5; the Qwen2.5 reading: untied E and W)    */
+/* ------------------------------------------------------------------------ */
+
+/* x[r] = E[tokens[r]] for M rows of H (bf16). tokens: device int32. A token
+ * outside [0, V) reads row 0 and increments *bad_tokens (device int32). */
+mt_status mt_embed_fwd(const int32_t* tokens, const mt_bf16* E, mt_bf16* x, int64_t M, int32_t H, int32_t V,
+                       int32_t* bad_tokens, void* stream);
+
+/* Host helper (no CUDA): the rows 0..M-1 stably sorted by token into order[M],
+ * and start[V+1] with token v's rows at order[start[v] .. start[v+1]). */
+mt_status mt_embed_sort(const int32_t* tokens, int64_t M, int32_t V, int32_t* order, int32_t* start);
+
+/* dE[v] = sum over token v's rows of dx (fp32 [V, H], every row written),
+ * added in increasing row order (bitwise repeatable). order/start: device
+ * copies of mt_embed_sort's output. */
+mt_status mt_embed_bwd(const int32_t* order, const int32_t* start, const mt_bf16* dx, float* dE, int32_t H, int32_t V,
+                       void* stream);
+
+/* Workspace of mt_head_loss_fwd_bwd. */
+uint64_t mt_head_workspace_bytes(int64_t M, int32_t H, int32_t V, int32_t vocab_chunk);
+
+/* Final RMSNorm (gain gf, eps) + LM head W [V, H] + mean cross-entropy over M
+ * rows of the stack output y against targets (device int32 in [0, V)), and its
+ * backward, over vocabulary chunks of vocab_chunk rows of W (the full logits
+ * never exist). Outputs: *loss (device fp32), dy [M, H] bf16, dgf [H] fp32,
+ * dW [V, H] fp32 (overwritten). H, V and vocab_chunk multiples of 8. */
+mt_status mt_head_loss_fwd_bwd(const mt_bf16* y, const mt_bf16* gf, const mt_bf16* W, const int32_t* targets,
+                               int64_t M, int32_t H, int32_t V, float eps, int32_t vocab_chunk, float* loss,
+                               mt_bf16* dy, float* dgf, float* dW, void* ws, uint64_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* CPU optimizer (blog summary, design point 1: the optimizer step runs on   */
 /* the CPU with Adam momentum and variance in host memory)                   */
 /* ------------------------------------------------------------------------ */

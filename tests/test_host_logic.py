@@ -172,3 +172,15 @@ def test_bench_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOPS" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_embedding_sort_is_stable_and_complete():
+    import numpy as np
+    tok = np.array([3, 1, 3, 0, 3, 1], np.int32)
+    order = np.empty(6, np.int32)
+    start = np.empty(5, np.int32)
+    L.mt_embed_sort(tok, 6, 4, order, start)
+    assert list(start) == [0, 1, 3, 3, 6]
+    assert list(order) == [3, 1, 5, 0, 2, 4]
+    with pytest.raises(L.MTError):
+        L.mt_embed_sort(np.array([4], np.int32), 1, 4, order, start)

@@ -58,6 +58,7 @@ ABLATIONS = {
     "no_slab_pool": {"no_slab_pool": 1},     # "w/o Gradient Slab Pool"
     "ckpt1": {"ckpt_interval": 1},           # "w/ Checkpoint Interval=1"
 }
+VOCAB = 152064  # Qwen2.5 tokenizer (an assumption: the pages do not state it)
 METRIC = "sustained TFLOPS (6ND+12LHT²) & tokens/s, streamed 7B/14B layer stack, 1 B200"
 UNIT = "TFLOPS"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -111,9 +112,12 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
     return units_per_rank * world / (ms_max / 1e3)
 
 
-def model_flops(cfg, p_layer):
+def model_flops(cfg, p_layer, vocab=0):
+    """6ND + 12LHT^2 with N the stack's parameters (plus the untied embedding and
+    LM head, 2 V H, for the whole model)."""
     sh = cfg["shape"]
-    return metrics.model_flops(cfg["L"] * p_layer, cfg["L"], sh["hidden"], cfg["B"], cfg["T"])
+    N = cfg["L"] * p_layer + 2 * vocab * sh["hidden"]
+    return metrics.model_flops(N, cfg["L"], sh["hidden"], cfg["B"], cfg["T"])
 
 
 # ---------------------------------------------------------------- clocks
@@ -326,7 +330,64 @@ def run_ours(args, cfg, rank, world, local_rank):
         return ms / steps
 
     dev_step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d, c_sink, sink_user)  # noqa: E731
+    head = None
+    if args.full_model:
+        # the whole model: embedding -> streamed stack -> final norm + LM head + loss (hook) -> streamed
+        # backward -> embedding gradient; E, W stay on the device, tokens are synthetic
+        V, chunk = VOCAB, 16384
+        M = B * T
+        g = torch.Generator(device="cuda").manual_seed(4321 + rank)
+        E_d = (torch.randn(V, H, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        W_d = (torch.randn(V, H, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        gf_d = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+        tok = np.random.default_rng(99 + rank).integers(0, V, size=M).astype(np.int32)
+        tok_d = torch.from_numpy(tok).cuda()
+        tgt_d = torch.from_numpy(np.roll(tok, -1).astype(np.int32)).cuda()
+        loss_d = torch.zeros(1, dtype=torch.float32, device="cuda")
+        dgf_d = torch.empty(H, dtype=torch.float32, device="cuda")
+        dWh_d = torch.empty(V, H, dtype=torch.float32, device="cuda")
+        dE_d = torch.empty(V, H, dtype=torch.float32, device="cuda")
+        bad_d = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nhw = L_.mt_head_workspace_bytes(M, H, V, chunk)
+        hws = torch.empty(nhw, dtype=torch.uint8, device="cuda")
+        order_h = torch.empty(M, dtype=torch.int32).pin_memory()
+        start_h = torch.empty(V + 1, dtype=torch.int32).pin_memory()
+        order_d = torch.empty(M, dtype=torch.int32, device="cuda")
+        start_d = torch.empty(V + 1, dtype=torch.int32, device="cuda")
+        tok_h = torch.from_numpy(tok).pin_memory()
+        loss_h = torch.zeros(1, dtype=torch.float32).pin_memory()
+
+        def hook(y_ptr, dy_ptr, stream, user):
+            try:
+                L_.mt_head_loss_fwd_bwd(y_ptr, gf_d, W_d, tgt_d, M, H, V, 1e-6, chunk, loss_d, dy_ptr, dgf_d, dWh_d,
+                                        hws, nhw, stream)
+                return 0
+            except L_.MTError as e:
+                return e.code
+
+        c_hook = L_.mt_head_hook(hook)
+        head = (c_hook, hws)  # keep the callback alive
+
+        def dev_step():
+            # host side of the embedding backward: the tokens' counting sort (the data loader's work)
+            L_.mt_embed_sort(tok_h, M, V, order_h, start_h)
+            with torch.cuda.stream(cs):
+                order_d.copy_(order_h, non_blocking=True)
+                start_d.copy_(start_h, non_blocking=True)
+                L_.mt_embed_fwd(tok_d, E_d, x_d, M, H, V, bad_d, cs)
+                L_.mt_stream_step_hooked(eng, store, x_d, dy_d, y_d, dx_d, c_sink, sink_user, c_hook, None)
+                L_.mt_embed_bwd(order_d, start_d, dx_d, dE_d, H, V, cs)
+
+        def full_host_step():  # tokens in from pinned host memory, the loss back out
+            with torch.cuda.stream(cs):
+                tok_d.copy_(tok_h, non_blocking=True)
+            dev_step()
+            with torch.cuda.stream(cs):
+                loss_h.copy_(loss_d, non_blocking=True)
+            cs.synchronize()
     host_step = lambda: L_.mt_stream_step_host(eng, store, xh, dyh, yh, dxh, c_sink, sink_user)  # noqa: E731
+    if args.full_model:
+        host_step = full_host_step
     for _ in range(args.warmup):
         dev_step()
     clocks = ClockSampler(local_rank)
@@ -341,7 +402,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     assert L_.mt_device_error(clear=True) == 0, "a kernel's bounded wait ran out"
     link = measure_link(torch) if rank == 0 else None
 
-    mflops = model_flops(cfg, p_layer)
+    mflops = model_flops(cfg, p_layer, VOCAB if args.full_model else 0)
     value = job_throughput(mflops, world, ms) / 1e12
     e2e = job_throughput(mflops, world, ms_e2e) / 1e12
     peaks, src = load_peaks()
@@ -362,6 +423,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg["name"], "layers": nL, "batch": B, "seq_len": T,
                        "ckpt_interval": abl.get("ckpt_interval", cfg["K"]), "ablation": args.ablation,
+                       "full_model": bool(args.full_model),
                        "mlp_chunk": cfg["chunk"], "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each layer's weights alone are %.0f MB)" % (p_layer * 2 / 1e6),
                        "sink": ("CPU AdamW on the fp32 master + bf16 refresh (library sink)" if args.sink == "adamw"
@@ -369,7 +431,8 @@ def run_ours(args, cfg, rank, world, local_rank):
             "tokens_per_s": B * T * world / (ms / 1e3),
             "clocks": clk,
             "e2e": {"value": e2e, "unit": UNIT,
-                    "h2d_bytes_per_step": int(st_e2e.h2d_bytes), "d2h_bytes_per_step": int(st_e2e.d2h_bytes)},
+                    "h2d_bytes_per_step": int(st_e2e.h2d_bytes) + ((2 * B * T + VOCAB + 1) * 4 if args.full_model else 0),
+                    "d2h_bytes_per_step": int(st_e2e.d2h_bytes) + (4 if args.full_model else 0)},
             "gpu_launches": int(st.kernel_launches) * args.steps,
             "roofline": {"bound": "tensor", "kernel": "gemm2_kernel (tcgen05, 2-SM)", "achieved": gemm_tf,
                          "peak": peak_tf, "unit": "TFLOP/s", "frac": (gemm_tf / peak_tf) if gemm_tf else None,
@@ -404,6 +467,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--full-model", action="store_true",
+                    help="add the embedding and the final norm + LM head + loss (vocabulary 152064) to the step")
     ap.add_argument("--sink", default="none", choices=["none", "adamw"],
                     help="what receives each layer's gradient record (adamw: the CPU optimizer step)")
     ap.add_argument("--ablation", default="none", choices=sorted(ABLATIONS),

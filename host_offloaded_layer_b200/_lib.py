@@ -61,6 +61,7 @@ class mt_adamw_cfg(ctypes.Structure):
 
 
 mt_grad_sink = ctypes.CFUNCTYPE(c_i32, c_i32, ctypes.POINTER(c_f32), c_u64, c_vp)
+mt_head_hook = ctypes.CFUNCTYPE(c_i32, c_vp, c_vp, c_vp, c_vp)
 
 _P = c_vp
 _CFG = ctypes.POINTER(mt_layer_cfg)
@@ -98,6 +99,7 @@ _SIGS = {
     "mt_engine_create": (c_i32, [_CFG, c_i32, c_i32, c_i32, ctypes.POINTER(mt_engine_opts), _P, c_u64, _P, _P, _P,
                                  ctypes.POINTER(c_vp)]),
     "mt_stream_step": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp]),
+    "mt_stream_step_hooked": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp, mt_head_hook, c_vp]),
     "mt_stream_step_host": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp]),
     "mt_engine_stats": (c_i32, [c_vp, ctypes.POINTER(mt_stats)]),
     "mt_engine_reset": (c_i32, [c_vp]),
@@ -305,6 +307,15 @@ _NULL_SINK = ctypes.cast(None, mt_grad_sink)
 def mt_stream_step(engine, store, x0, dy_top, y_top, dx0, sink=None, user=None):
     _check(load().mt_stream_step(engine, store, _ptr(x0), _ptr(dy_top), _ptr(y_top), _ptr(dx0),
                                  sink if sink is not None else _NULL_SINK, user))
+
+
+_NULL_HOOK = ctypes.cast(None, mt_head_hook)
+
+
+def mt_stream_step_hooked(engine, store, x0, dy_top, y_top, dx0, sink=None, user=None, hook=None, hook_user=None):
+    _check(load().mt_stream_step_hooked(engine, store, _ptr(x0), _ptr(dy_top), _ptr(y_top), _ptr(dx0),
+                                        sink if sink is not None else _NULL_SINK, user,
+                                        hook if hook is not None else _NULL_HOOK, hook_user))
 
 
 def mt_stream_step_host(engine, store, x0, dy_top, y_top, dx0, sink=None, user=None):

@@ -348,7 +348,7 @@ void prepare_schedule(mt_engine* e) {
 }
 
 mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top, mt_bf16* y_top,
-                   mt_bf16* dx0, mt_grad_sink sink, void* user) {
+                   mt_bf16* dx0, mt_grad_sink sink, void* user, mt_head_hook hook, void* hook_user) {
   const uint64_t rec = e->G.off.record_elems;
   const int n = static_cast<int>(e->uses.size());
   const bool skip_loads = e->opts.resident && e->resident_loaded;
@@ -408,6 +408,11 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
     status = enqueue_loads(i);
     if (status != MT_OK) break;
     const Use u = e->uses[i];
+    if (hook && u.kind != 0 && e->uses[i - 1].kind == 0) {
+      // between the forward and the backward: the caller's head turns y_top into dy_top
+      status = hook(y_top, const_cast<mt_bf16*>(dy_top), e->cs, hook_user);
+      if (status != MT_OK) break;
+    }
     const int l = u.layer;
     const int s = l / e->K, a = s * e->K;
     mt_bf16* w = e->slot[e->uslot[i]];
@@ -611,6 +616,12 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
 
 mt_status mt_stream_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top, mt_bf16* y_top,
                          mt_bf16* dx0, mt_grad_sink sink, void* user) {
+  return mt_stream_step_hooked(e, store, x0, const_cast<mt_bf16*>(dy_top), y_top, dx0, sink, user, nullptr, nullptr);
+}
+
+mt_status mt_stream_step_hooked(mt_engine* e, mt_host_store* store, const mt_bf16* x0, mt_bf16* dy_top,
+                                mt_bf16* y_top, mt_bf16* dx0, mt_grad_sink sink, void* user, mt_head_hook hook,
+                                void* hook_user) {
   if (!e || !store || !x0 || !dy_top || !y_top || !dx0) return fail(MT_ERR_INVALID_ARG, "stream_step: NULL argument");
   if (store->L != e->L || store->G.off.record_elems != e->G.off.record_elems)
     return fail(MT_ERR_INVALID_ARG, "host store does not match the engine's layer count or shape");
@@ -629,7 +640,7 @@ mt_status mt_stream_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, 
   e->timer.flops.clear();
   e->timer.overflow = false;
   if (e->opts.time_gemms) set_gemm_timer(&e->timer);
-  mt_status s = run_step(e, store, x0, dy_top, y_top, dx0, sink, user);
+  mt_status s = run_step(e, store, x0, dy_top, y_top, dx0, sink, user, hook, hook_user);
   set_gemm_timer(nullptr);
   e->st.step_ms = std::chrono::duration<double, std::milli>(Clock::now() - t0).count();
   e->st.exec_flops = exec_flops_counter() - f0;

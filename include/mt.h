@@ -313,6 +313,18 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
 mt_status mt_stream_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top,
                          mt_bf16* y_top, mt_bf16* dx0, mt_grad_sink sink, void* user);
 
+/* Called on the enqueuing thread once per step, after the last layer's
+ * forward has been enqueued and before the first backward work: enqueue, on
+ * compute_stream, whatever turns y_top into dy_top (a final norm, LM head and
+ * loss, for instance). Return MT_OK to continue the step. */
+typedef mt_status (*mt_head_hook)(const mt_bf16* y_top, mt_bf16* dy_top, void* compute_stream, void* user);
+
+/* mt_stream_step with a head between forward and backward: when hook is not
+ * NULL, dy_top is written by the hook instead of being an input. */
+mt_status mt_stream_step_hooked(mt_engine* e, mt_host_store* store, const mt_bf16* x0, mt_bf16* dy_top,
+                                mt_bf16* y_top, mt_bf16* dx0, mt_grad_sink sink, void* user, mt_head_hook hook,
+                                void* hook_user);
+
 /* Same step with x0/dy_top/y_top/dx0 in host memory (pinned for full speed):
  * the inputs are copied in and the outputs copied out inside the call. */
 mt_status mt_stream_step_host(mt_engine* e, mt_host_store* store, const mt_bf16* x0_host,

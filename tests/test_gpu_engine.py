@@ -240,3 +240,76 @@ def test_cpu_optimizer_sink_closes_the_training_loop():
     finally:
         L.mt_host_optimizer_destroy(opt)
         s.close()
+
+
+def test_full_model_step_with_embedding_and_head_hook():
+    """Embedding -> streamed layer stack -> (hook) final norm + LM head + loss ->
+    streamed backward -> embedding gradient, against the oracle end to end."""
+    import torch
+
+    from oracle import head as HD
+    V, Lyr, B, T = 1000, 2, 2, 128
+    s = Stack(TINY, Lyr, B, T, ckpt_interval=2)
+    try:
+        Hd = TINY["hidden"]
+        M = B * T
+        rng = np.random.default_rng(17)
+        tok = rng.integers(0, V, size=M).astype(np.int32)
+        tgt = np.roll(tok, -1).astype(np.int32)
+        E = synth.f32_to_bf16_bits(synth.normal_f32(3, 0, 1, V * Hd, 1.0)).reshape(V, Hd)
+        W = synth.f32_to_bf16_bits(synth.normal_f32(3, 0, 2, V * Hd, 0.05)).reshape(V, Hd)
+        gf = synth.f32_to_bf16_bits(np.ones(Hd, np.float32))
+        E_d, W_d, gf_d = H.dev_bf16(E), H.dev_bf16(W), H.dev_bf16(gf)
+        tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+        x0 = H.empty_bf16(B, T, Hd)
+        bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+        L.mt_embed_fwd(tok_d, E_d, x0, M, Hd, V, bad)
+        loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+        dgf = H.empty_f32(Hd)
+        dWh = H.empty_f32(V, Hd)
+        chunk = 384
+        ws = H.workspace(L.mt_head_workspace_bytes(M, Hd, V, chunk))
+
+        def hook(y_ptr, dy_ptr, stream, user):
+            try:
+                L.mt_head_loss_fwd_bwd(y_ptr, gf_d, W_d, tgt_d, M, Hd, V, 1e-6, chunk, loss, dy_ptr, dgf, dWh, ws,
+                                       ws.numel(), stream)
+                return 0
+            except L.MTError as e:
+                return e.code
+
+        c_hook = L.mt_head_hook(hook)
+        y = H.empty_bf16(B, T, Hd)
+        dy = H.empty_bf16(B, T, Hd)
+        dx0 = H.empty_bf16(B, T, Hd)
+        torch.cuda.synchronize()
+        s.grads = {}
+        L.mt_stream_step_hooked(s.eng, s.store, x0, dy, y, dx0, s.sink, None, c_hook, None)
+        order = np.empty(M, np.int32)
+        start = np.empty(V + 1, np.int32)
+        L.mt_embed_sort(tok, M, V, order, start)
+        dE = H.empty_f32(V, Hd)
+        L.mt_embed_bwd(torch.from_numpy(order).cuda(), torch.from_numpy(start).cuda(), dx0, dE, Hd, V)
+        torch.cuda.synchronize()
+        assert L.mt_device_error(clear=True) == 0 and bad.item() == 0
+        # the oracle, end to end
+        ocfg = H.oracle_cfg(s.cfg)
+        x64 = HD.embed_fwd(tok.reshape(B, T), H.bits_to_f64(E))
+        yy = x64
+        for w in s.w64:
+            yy, _ = O.layer_fwd(ocfg, w, yy)
+        l_ref, dy_ref, dgf_ref, dW_ref = HD.head_loss_fwd_bwd(yy, H.bits_to_f64(gf), H.bits_to_f64(W),
+                                                              tgt.reshape(B, T), 1e-6)
+        _, dx_ref, g_ref = O.stack_fwd_bwd(ocfg, s.w64, x64, dy_ref)
+        dE_ref = HD.embed_bwd(tok.reshape(B, T), dx_ref, V)
+        assert abs(loss.item() - l_ref) / l_ref < 1e-3
+        assert H.rel(H.host_f64(dy), dy_ref) < H.TOL
+        assert H.rel(H.host_f64(dWh), dW_ref) < H.TOL and H.rel(H.host_f64(dgf), dgf_ref) < H.TOL
+        assert H.rel(H.host_f64(dx0), dx_ref) < H.TOL
+        assert H.rel(H.host_f64(dE), dE_ref) < H.TOL
+        for l in range(Lyr):
+            got = H.grads_from_record(s.cfg, s.grads[l])
+            for k, v in g_ref[l].items():
+                assert H.rel(got[k], v) < H.TOL, (l, k)
+    finally:
+        s.close()

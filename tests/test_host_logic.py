@@ -21,8 +21,9 @@ TINY = dict(hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=688)
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "mt.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"\b(mt_[a-z0-9_]+)\s*\(", src)
-    return sorted(set(n for n in names if n != "mt_grad_sink"))
+    # function declarations: a return type, the name, "(" (function-pointer typedefs are "(*name)")
+    names = re.findall(r"\b(?:mt_status|uint64_t|int32_t|void|float|mt_bf16|char)\s*\*?\s*(mt_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
 
 
 def test_library_exports_every_declared_entry_point(lib):

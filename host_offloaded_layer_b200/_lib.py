@@ -77,6 +77,7 @@ _SIGS = {
     "mt_gemm_bf16": (c_i32, [_P, c_i64, c_i32, _P, c_i64, c_i32, _P, c_i64, c_i32, c_i32, c_i64, c_i64, c_i64,
                              _P, _P, c_i64, _P]),
     "mt_gemm_swiglu_bf16": (c_i32, [_P, c_i64, _P, c_i64, _P, c_i64, _P, c_i64, c_i64, c_i64, c_i64, _P]),
+    "mt_gemm_swiglu_bwd_bf16": (c_i32, [_P, c_i64, _P, c_i64, _P, c_i64, c_i64, c_i64, c_i64, _P]),
     "mt_rmsnorm_fwd": (c_i32, [_P, _P, _P, _P, c_i64, c_i32, c_f32, _P]),
     "mt_rmsnorm_bwd_workspace_bytes": (c_u64, [c_i64, c_i32]),
     "mt_rmsnorm_bwd": (c_i32, [_P, _P, _P, _P, _P, _P, _P, c_i64, c_i32, _P, c_u64, _P]),
@@ -209,6 +210,10 @@ def mt_gemm_bf16(A, lda, a_mn_major, Bm, ldb, b_mn_major, C, ldc, c_f32, accumul
 def mt_gemm_swiglu_bf16(A, lda, Wgu, ldw, m, ldm, gu, ld_gu, M, F, K, stream=None):
     _check(load().mt_gemm_swiglu_bf16(_ptr(A), lda, _ptr(Wgu), ldw, _ptr(m), ldm, _ptr(gu), ld_gu, M, F, K,
                                       _stream(stream)))
+
+
+def mt_gemm_swiglu_bwd_bf16(dY, ld_dy, Wd, ldw, gu, ld_gu, M, F, K, stream=None):
+    _check(load().mt_gemm_swiglu_bwd_bf16(_ptr(dY), ld_dy, _ptr(Wd), ldw, _ptr(gu), ld_gu, M, F, K, _stream(stream)))
 
 
 def mt_rmsnorm_fwd(x, g, y, rstd, rows, H, eps, stream=None):

@@ -2,21 +2,28 @@
 // (head_dim 128): S = Q K^T and O += P V are tcgen05.mma with both
 // accumulators in tensor memory, the operands staged by TMA.
 //
-// One CTA per (128 query rows, query head, sequence):
-//   warp 0     TMA: Q once, then K_j and V_j (128 key rows each) into a
-//              two-stage ring;
+// Persistent: one CTA per SM walks the (128 query rows, query head, sequence)
+// tiles, longest rows first, so the next tile's Q load and first two S MMAs
+// overlap the current tile's output epilogue.
+//   warp 0     TMA: lane 0 loads Q per tile and K_j, lane 1 V_j (128 key
+//              rows each), each into its own two-stage ring: a K stage is
+//              free once S_j is done, a V stage once O += P_j V_j is;
 //   warp 1     TMEM allocation and the MMA issuer: S_{j+1} = Q K_{j+1}^T is
 //              issued before O += P_j V_j so the tensor cores work while the
 //              softmax of block j runs;
-//   warps 2-5  softmax, one thread per query row: S row from TMEM, online
-//              softmax in the log2 domain, P (bf16) written to shared memory
-//              in the 128-byte-swizzled K-major layout the next MMA reads,
-//              then the final O / l and the log-sum-exp.
-// TMEM: two S buffers (128 columns each) and O (128 columns). O is rescaled
-// only when a row's running maximum grows by more than 8 (a factor 256 in
-// the exponent); otherwise the stale maximum stays, which keeps P <= 256 and
-// the result exact up to rounding (the final division uses the same
-// maximum as every P). Every mbarrier wait is bounded.
+//   warps 2-9  softmax in two groups of four warps, one thread per query row
+//              and group. Group g owns key columns [64 g, 64 g + 64) of every
+//              block and its own output accumulator O_g = sum_j P_j,g V_j,g
+//              with its own running maximum and sum (a split of the key axis
+//              inside the CTA), so the groups never synchronise inside the
+//              key loop; the two partial results meet once per tile:
+//              O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)).
+// Scores are handled in the log2 domain. TMEM: two S buffers (128 columns
+// each), O_0 and O_1 (128 columns each). O_g is rescaled only when its row
+// maximum grows by more than 8 (a factor 256 in the exponent); otherwise the
+// stale maximum stays, which keeps P <= 256 and the result exact up to
+// rounding (the final combination uses the same maxima as every P). Every
+// mbarrier wait is bounded.
 #include <mutex>
 
 #include "mt_internal.h"
@@ -33,18 +40,33 @@ constexpr int ATOM = 128 * 64 * 2;  // 16 KiB
 // shared memory: Q | K0 V0 | K1 V1 | P0 | P1
 constexpr int OFF_Q = 0, OFF_KV = TILE, OFF_P = 5 * TILE;
 constexpr int SMEM_TILES = 7 * TILE;
-constexpr int SMEM_BYTES = SMEM_TILES + 128 + 1024 + 1024;  // tiles, barriers, row exchange, alignment
+constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;  // tiles, barriers, alignment
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S0 = 0, COL_O = 256;
+constexpr uint32_t COL_S0 = 0, COL_O = 256;  // S_s at 128 s, O_g at 256 + 128 g
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
+constexpr int FWD_THREADS = 64 + 256;
 
-// Bounded barrier among a group of threads built on an mbarrier initialised
-// with the group's size: arrive, then wait (bounded) for the phase to flip.
-// `phase` counts this thread's uses. Returns false when the wait ran out.
-__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag, int32_t* err) {
-  mbar_arrive(bar);
+// 2^x by the MUFU instruction (flush-to-zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One arrival per warp: the warp's lanes are ordered by __syncwarp, then
+// lane 0 arrives (release) on behalf of all of them.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Bounded barrier among groups of warps on an mbarrier initialised with the
+// number of warps: arrive once per warp, then every thread waits for the phase
+// to flip. `phase` counts this thread's uses. Returns false when the wait ran out.
+__device__ __forceinline__ bool warps_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag, int32_t* err) {
+  warp_arrive(bar);
   const bool ok = mbar_wait(bar, phase & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE);
   ++phase;
   return ok;
@@ -55,47 +77,59 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// NG softmax warpgroups: with NG = 2, warps 2-5 take key columns 0-63 (and O
-// columns 0-63) of the 128 rows, warps 6-9 columns 64-127 of the same rows;
-// the two halves of each row maximum and row sum meet in shared memory.
-template <int NG>
-__global__ void __launch_bounds__(64 + 128 * NG, 1)
+// Tile t of the persistent walk: query blocks from the last (longest rows)
+// down, then query head, then sequence.
+struct FwdTile {
+  int qb, h, b;
+};
+__device__ __forceinline__ FwdTile fwd_tile(int t, int n_qb, int nq, int B) {
+  const int per_qb = nq * B;
+  const int rest = t % per_qb;
+  return {n_qb - 1 - t / per_qb, rest % nq, rest / nq};
+}
+
+__global__ void __launch_bounds__(FWD_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16* __restrict__ o, int64_t ld_o,
-                       float* __restrict__ lse, int T, int nq, int nkv, float scale_log2, int32_t* err) {
-  constexpr int SCOLS = BKV / NG, OCOLS = D / NG;  // S and O columns per softmax group
+                       float* __restrict__ lse, int B, int T, int nq, int nkv, float scale_log2, int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
-  uint64_t* q_full = bars;          // 1
-  uint64_t* kv_full = bars + 1;     // 2
-  uint64_t* kv_empty = bars + 3;    // 2
-  uint64_t* s_full = bars + 5;      // 2
-  uint64_t* p_full = bars + 7;      // 2
-  uint64_t* o_done = bars + 9;      // 2
-  uint64_t* x_bar = bars + 11;      // 1: row exchange between the softmax groups
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* q_full = bars;        // 1: Q of the tile loaded
+  uint64_t* q_empty = bars + 1;   // 1: the tile's S MMAs (the readers of Q) are done
+  uint64_t* k_full = bars + 2;    // 2
+  uint64_t* k_empty = bars + 4;   // 2
+  uint64_t* v_full = bars + 6;    // 2
+  uint64_t* v_empty = bars + 8;   // 2
+  uint64_t* s_full = bars + 10;   // 2
+  uint64_t* p_full = bars + 12;   // [group][buffer]: 4, one arrival per warp of the group
+  uint64_t* o_done = bars + 16;   // [group][buffer]: 4
+  uint64_t* o_free = bars + 20;   // 1: the tile's O accumulators have been read (8 warps)
+  uint64_t* x_bar = bars + 21;    // 1: row exchange between the groups (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xch = reinterpret_cast<float*>(smem + SMEM_TILES + 128);  // [NG][128] row halves
+  // the groups' row maxima and sums meet in P buffer 0, which is idle by then: [m | l][group][128 rows]
+  float* xch = reinterpret_cast<float*>(smem + OFF_P);
 
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int c = (h * nkv) / nq;
-  const int q0 = qb * BQ;
-  const int n_kv = min((T + BKV - 1) / BKV, qb + 1);
+  const int n_qb = (T + BQ - 1) / BQ;
+  const int n_tiles = n_qb * nq * B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = b * T;  // first row of this sequence in the [B*T, ld] qkv array
-  const int col_q = h * D, col_k = (nq + c) * D, col_v = (nq + nkv + c) * D;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
+    mbar_init(smem_u32(q_empty), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&kv_full[i]), 1);
-      mbar_init(smem_u32(&kv_empty[i]), 1);
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), 128 * NG);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&p_full[i]), 4);
       mbar_init(smem_u32(&o_done[i]), 1);
     }
-    mbar_init(smem_u32(x_bar), 128 * NG);
+    mbar_init(smem_u32(o_free), 8);
+    mbar_init(smem_u32(x_bar), 8);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
@@ -112,39 +146,51 @@ __global__ void __launch_bounds__(64 + 128 * NG, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint32_t qb_bar = smem_u32(q_full);
-      mbar_expect_tx(qb_bar, TILE);
-      tma_load_2d(smem_u32(smem + OFF_Q), &tm_qkv, qb_bar, col_q, row0 + q0);
-      tma_load_2d(smem_u32(smem + OFF_Q + ATOM), &tm_qkv, qb_bar, col_q + 64, row0 + q0);
+    // ------------------------------------------------------------ TMA producer (lane 0: Q, K; lane 1: V)
+    if (lane < 2) {
+      uint32_t it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+        const FwdTile w = fwd_tile(t, n_qb, nq, B);
+        const int c = (w.h * nkv) / nq;
+        const int row0 = w.b * T, q0 = w.qb * BQ;
+        const int n_kv = min(n_qb, w.qb + 1);
+        if (lane == 0) {
+          if (tl > 0 && !mbar_wait(smem_u32(q_empty), (tl - 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          const uint32_t qb_bar = smem_u32(q_full);
+          const int col_q = w.h * D;
+          mbar_expect_tx(qb_bar, TILE);
+          tma_load_2d(smem_u32(smem + OFF_Q), &tm_qkv, qb_bar, col_q, row0 + q0);
+          tma_load_2d(smem_u32(smem + OFF_Q + ATOM), &tm_qkv, qb_bar, col_q + 64, row0 + q0);
+        }
+        const int col = lane == 0 ? (nq + c) * D : (nq + nkv + c) * D;  // K or V columns
+        uint64_t* full = lane == 0 ? k_full : v_full;
+        uint64_t* empty = lane == 0 ? k_empty : v_empty;
+        const int off = lane == 0 ? 0 : TILE;
+        for (int j = 0; j < n_kv; ++j, ++it) {
+          const int s = it & 1;
+          if (!mbar_wait(smem_u32(&empty[s]), ((it >> 1) & 1u) ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[s]);
+          uint8_t* dst = smem + OFF_KV + s * 2 * TILE + off;
+          const int r = row0 + j * BKV;
+          mbar_expect_tx(fb, TILE);
+          tma_load_2d(smem_u32(dst), &tm_qkv, fb, col, r);
+          tma_load_2d(smem_u32(dst + ATOM), &tm_qkv, fb, col + 64, r);
+        }
+      }
     }
     __syncwarp();
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j & 1;
-      if (!warp_wait(smem_u32(&kv_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
-      if (lane == 0) {
-        const uint32_t fb = smem_u32(&kv_full[s]);
-        uint8_t* kt = smem + OFF_KV + s * 2 * TILE;
-        uint8_t* vt = kt + TILE;
-        const int r = row0 + j * BKV;
-        mbar_expect_tx(fb, 2 * TILE);
-        tma_load_2d(smem_u32(kt), &tm_qkv, fb, col_k, r);
-        tma_load_2d(smem_u32(kt + ATOM), &tm_qkv, fb, col_k + 64, r);
-        tma_load_2d(smem_u32(vt), &tm_qkv, fb, col_v, r);
-        tma_load_2d(smem_u32(vt + ATOM), &tm_qkv, fb, col_v + 64, r);
-      }
-      __syncwarp();
-    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, BKV, false, false);  // S = Q K^T: both K-major
-    constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);     // O += P V: V is MN-major (d contiguous)
+    constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);     // O_g += P_g V_g: V is MN-major (d contiguous)
     const uint32_t q_base = smem_u32(smem + OFF_Q);
-    bool ok = warp_wait(smem_u32(q_full), 0, abort_flag, err, DEV_ERR_TIMEOUT_MMA);
-    auto issue_s = [&](int j) -> bool {
-      const int s = j & 1;
-      if (!warp_wait(smem_u32(&kv_full[s]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
+    auto issue_s = [&](uint32_t i) -> bool {
+      const int s = i & 1;
+      if (!warp_wait(smem_u32(&k_full[s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
       fence_after();
       if (lane == 0) {
         const uint32_t k_base = smem_u32(smem + OFF_KV + s * 2 * TILE);
@@ -155,166 +201,204 @@ __global__ void __launch_bounds__(64 + 128 * NG, 1)
                     idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(smem_u32(&s_full[s]));
+        umma_commit(smem_u32(&k_empty[s]));
       }
       __syncwarp();
       return true;
     };
-    if (ok) ok = issue_s(0);
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int s = j & 1;
-      if (j + 1 < n_kv && !issue_s(j + 1)) break;
-      if (!warp_wait(smem_u32(&p_full[s]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
-      fence_after();
-      if (lane == 0) {
+    uint32_t it = 0, tl = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      const FwdTile w = fwd_tile(t, n_qb, nq, B);
+      const int n_kv = min(n_qb, w.qb + 1);
+      if (!warp_wait(smem_u32(q_full), tl & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA) || !issue_s(it)) break;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const uint32_t i = it + j;
+        const int s = i & 1;
+        if (j + 1 < n_kv) {
+          if (!issue_s(i + 1)) {
+            ok = false;
+            break;
+          }
+        } else {
+          if (lane == 0) umma_commit(smem_u32(q_empty));  // every S MMA of the tile is issued
+          __syncwarp();
+        }
+        // the first P V of a tile overwrites O: the previous tile's epilogue must have read it
+        if (j == 0 && tl > 0 && !warp_wait(smem_u32(o_free), (tl - 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
         const uint32_t p_base = smem_u32(smem + OFF_P + s * TILE);
         const uint32_t v_base = smem_u32(smem + OFF_KV + s * 2 * TILE + TILE);
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint32_t poff = static_cast<uint32_t>((kk >> 2) * ATOM + (kk & 3) * 32);
-          umma_bf16(tmem + COL_O, smem_desc(p_base + poff, 16, 1024), smem_desc(v_base + kk * 2048, ATOM, 1024),
-                    idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(smem_u32(&o_done[s]));
-        umma_commit(smem_u32(&kv_empty[s]));
-      }
-      __syncwarp();
-    }
-  } else {
-    // ------------------------------------------------------------ softmax (one thread per query row and group)
-    const int g = (warp - 2) >> 2;  // softmax group: columns [g*SCOLS, (g+1)*SCOLS) of S
-    const int qw = warp & 3;        // TMEM lanes [32 qw, 32 qw + 32)
-    const int r = qw * 32 + lane;
-    const int q_row = q0 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
-    uint32_t xph = 0;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j & 1;
-      if (!warp_wait(smem_u32(&s_full[s]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      float sv[SCOLS];
-#pragma unroll
-      for (int ch = 0; ch < SCOLS / 32; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + COL_S0 + s * BKV + g * SCOLS + ch * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
-      }
-      const int k0 = j * BKV + g * SCOLS;
-      const bool diag = k0 + SCOLS - 1 > q0;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < SCOLS; ++e) {
-        float v = sv[e] * scale_log2;
-        if (diag && k0 + e > q_row) v = -INFINITY;
-        sv[e] = v;
-        mx = fmaxf(mx, v);
-      }
-      if (NG == 2) {  // the other half of the row's maximum
-        xch[g * 128 + r] = mx;
-        if (!group_sync(smem_u32(x_bar), xph, abort_flag, err)) {
+        if (!warp_wait(smem_u32(&v_full[s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
-        mx = fmaxf(mx, xch[(g ^ 1) * 128 + r]);
-        if (!group_sync(smem_u32(x_bar), xph, abort_flag, err)) {  // both halves read before the next write
-          ok = false;
-          break;
-        }
-      }
-      // rescale O only when some row of the warp raised its maximum by more than the threshold
-      // (the decision is the same in both groups: it depends on the row maximum only)
-      const bool need = (m_run == -INFINITY) || (mx > m_run + RESCALE_THRESHOLD);
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = exp2f(m_run - m_new);  // 0 for the first block
-        if (j > 0) {
-          // O must hold P_{j-1} V_{j-1} before it is rescaled
-          if (!warp_wait(smem_u32(&o_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_flag, err,
-                         DEV_ERR_TIMEOUT_EPILOGUE)) {
+        for (int g = 0; g < 2; ++g) {
+          if (!warp_wait(smem_u32(&p_full[g * 2 + s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
             ok = false;
             break;
           }
           fence_after();
+          if (lane == 0) {
 #pragma unroll
-          for (int ch = 0; ch < OCOLS / 32; ++ch) {
-            uint32_t u[32];
-            const uint32_t col = COL_O + g * OCOLS + ch * 32;
-            tmem_ld32(tmem + lane_base + col, u);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(tmem + lane_base + col, u);
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_bf16(tmem + COL_O + g * D, smem_desc(p_base + g * ATOM + kk * 32, 16, 1024),
+                        smem_desc(v_base + (g * 4 + kk) * 2048, ATOM, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&o_done[g * 2 + s]));
+            if (g == 1) umma_commit(smem_u32(&v_empty[s]));
           }
+          __syncwarp();
         }
-        l_run *= alpha;
-        m_run = m_new;
       }
-      // P_{j-2} V_{j-2} must be done reading P buffer s before it is overwritten
-      if (j >= 2) {
-        if (!warp_wait(smem_u32(&o_done[s]), ((j - 2) >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
+      it += n_kv;
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (one thread per query row and group)
+    const int g = (warp - 2) >> 2;  // key columns [64 g, 64 g + 64) of every block, accumulator O_g
+    const int qw = warp & 3;        // TMEM lanes [32 qw, 32 qw + 32)
+    const int r = qw * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
+    const uint32_t col_og = COL_O + g * D;
+    uint32_t it = 0, tl = 0, xph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      const FwdTile w = fwd_tile(t, n_qb, nq, B);
+      const int q0 = w.qb * BQ, q_row = q0 + r, row0 = w.b * T;
+      const int n_kv = min(n_qb, w.qb + 1);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < n_kv; ++j) {
+        const uint32_t i = it + j;
+        const int s = i & 1;
+        if (!warp_wait(smem_u32(&s_full[s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
           ok = false;
           break;
         }
-      }
-      uint8_t* prow = smem + OFF_P + s * TILE + r * 128;
-      float lsum = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < SCOLS / 8; ++ch) {  // 16-byte chunks of 8 columns
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(sv[ch * 8 + e] - m_run);
-          lsum += p[e];
-        }
-        uint4 w;
-        w.x = pack_bf16(p[0], p[1]);
-        w.y = pack_bf16(p[2], p[3]);
-        w.z = pack_bf16(p[4], p[5]);
-        w.w = pack_bf16(p[6], p[7]);
-        const int cg = g * (SCOLS / 8) + ch;  // chunk index within the row of 128 columns
-        const int atom = cg >> 3, c16 = cg & 7;
-        *reinterpret_cast<uint4*>(prow + atom * ATOM + ((c16 ^ (r & 7)) << 4)) = w;
-      }
-      l_run += lsum;
-      fence_proxy_async_smem();
-      fence_before();
-      mbar_arrive(smem_u32(&p_full[s]));
-    }
-    float l_tot = l_run;
-    if (NG == 2 && ok) {
-      xch[g * 128 + r] = l_run;
-      ok = group_sync(smem_u32(x_bar), xph, abort_flag, err);
-      l_tot = l_run + xch[(g ^ 1) * 128 + r];
-    }
-    if (ok && n_kv > 0) {
-      const int jl = n_kv - 1;
-      if (warp_wait(smem_u32(&o_done[jl & 1]), (jl >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
         fence_after();
-        const float inv = 1.f / l_tot;
-        __nv_bfloat16* orow = o + (static_cast<int64_t>(row0) + q_row) * ld_o + static_cast<int64_t>(h) * D;
+        float sv[64];
 #pragma unroll
-        for (int ch = 0; ch < OCOLS / 32; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t u[32];
-          const int oc = g * OCOLS + ch * 32;
-          tmem_ld32(tmem + lane_base + COL_O + oc, u);
-          if (q_row < T) {
+          tmem_ld32(tmem + lane_base + COL_S0 + s * BKV + g * 64 + ch * 32, u);
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(u[qd * 8 + 0]) * inv, __uint_as_float(u[qd * 8 + 1]) * inv);
-              w.y = pack_bf16(__uint_as_float(u[qd * 8 + 2]) * inv, __uint_as_float(u[qd * 8 + 3]) * inv);
-              w.z = pack_bf16(__uint_as_float(u[qd * 8 + 4]) * inv, __uint_as_float(u[qd * 8 + 5]) * inv);
-              w.w = pack_bf16(__uint_as_float(u[qd * 8 + 6]) * inv, __uint_as_float(u[qd * 8 + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + oc + qd * 8) = w;
+          for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
+        }
+        const int k0 = j * BKV + g * 64;
+        float mx = -INFINITY;
+        if (k0 + 63 > q0) {  // a block on the diagonal: keys after the row are masked
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            if (k0 + e > q_row) sv[e] = -INFINITY;
+            mx = fmaxf(mx, sv[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, sv[e]);
+        }
+        mx *= scale_log2;
+        // rescale O_g only when some row of the warp raised its maximum by more than the threshold
+        if (__any_sync(0xffffffffu, mx > m_run + RESCALE_THRESHOLD)) {
+          const float m_new = fmaxf(m_run, mx);
+          const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run - m_new);  // 0 while m_run = -inf
+          if (j > 0) {
+            // O_g must hold P_{j-1} V_{j-1} before it is rescaled
+            const uint32_t ip = i - 1;
+            if (!warp_wait(smem_u32(&o_done[g * 2 + (ip & 1)]), (ip >> 1) & 1u, abort_flag, err,
+                           DEV_ERR_TIMEOUT_EPILOGUE)) {
+              ok = false;
+              break;
+            }
+            fence_after();
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t u[32];
+              tmem_ld32(tmem + lane_base + col_og + ch * 32, u);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+              tmem_st32(tmem + lane_base + col_og + ch * 32, u);
             }
           }
+          l_run *= alpha;
+          m_run = m_new;
         }
-        if (q_row < T && g == 0) lse[(static_cast<int64_t>(b) * nq + h) * T + q_row] = (m_run + log2f(l_tot)) * LN2;
+        // P V of block i - 2 must be done reading this group's half of P buffer s
+        if (i >= 2 && !warp_wait(smem_u32(&o_done[g * 2 + s]), ((i - 2) >> 1) & 1u, abort_flag, err,
+                                 DEV_ERR_TIMEOUT_EPILOGUE)) {
+          ok = false;
+          break;
+        }
+        const float mb = m_run == -INFINITY ? 0.f : m_run;  // a fully masked row half gives P = 0
+        uint8_t* prow = smem + OFF_P + s * TILE + g * ATOM + r * 128;
+        float lsum = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunks of 8 columns
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = ex2(fmaf(sv[ch * 8 + e], scale_log2, -mb));
+            lsum += p[e];
+          }
+          uint4 wv;
+          wv.x = pack_bf16(p[0], p[1]);
+          wv.y = pack_bf16(p[2], p[3]);
+          wv.z = pack_bf16(p[4], p[5]);
+          wv.w = pack_bf16(p[6], p[7]);
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = wv;
+        }
+        l_run += lsum;
+        fence_proxy_async_smem();
+        fence_before();
+        warp_arrive(smem_u32(&p_full[g * 2 + s]));
       }
+      if (!ok) break;
+      it += n_kv;
+      // ---- the two groups' partial results meet: O = (O_0 f_0 + O_1 f_1) / l. Both groups' last
+      // P V are done first, so O is final and neither P buffer is read any more.
+      const uint32_t il = it - 1;
+      if (!warp_wait(smem_u32(&o_done[il & 1]), (il >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE) ||
+          !warp_wait(smem_u32(&o_done[2 + (il & 1)]), (il >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      xch[g * 128 + r] = m_run;
+      xch[256 + g * 128 + r] = l_run;
+      if (!warps_sync(smem_u32(x_bar), xph, abort_flag, err)) break;
+      const float m_o = xch[(g ^ 1) * 128 + r], l_o = xch[256 + (g ^ 1) * 128 + r];
+      if (!warps_sync(smem_u32(x_bar), xph, abort_flag, err)) break;  // both read before P is written again
+      const float m = fmaxf(m_run, m_o);
+      const float f_self = ex2(m_run - m), f_other = ex2(m_o - m);
+      const float inv = 1.f / (l_run * f_self + l_o * f_other);
+      const float f0 = g == 0 ? f_self : f_other, f1 = g == 0 ? f_other : f_self;
+      __nv_bfloat16* orow = o + (static_cast<int64_t>(row0) + q_row) * ld_o + static_cast<int64_t>(w.h) * D;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {  // this group writes output columns [64 g, 64 g + 64)
+        const int oc = g * 64 + ch * 32;
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tmem + lane_base + COL_O + oc, u0);
+        tmem_ld32(tmem + lane_base + COL_O + D + oc, u1);
+        if (q_row < T) {
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              v[e] = (__uint_as_float(u0[qd * 8 + e]) * f0 + __uint_as_float(u1[qd * 8 + e]) * f1) * inv;
+            uint4 wv;
+            wv.x = pack_bf16(v[0], v[1]);
+            wv.y = pack_bf16(v[2], v[3]);
+            wv.z = pack_bf16(v[4], v[5]);
+            wv.w = pack_bf16(v[6], v[7]);
+            *reinterpret_cast<uint4*>(orow + oc + qd * 8) = wv;
+          }
+        }
+      }
+      if (q_row < T && g == 0)
+        lse[(static_cast<int64_t>(w.b) * nq + w.h) * T + q_row] = (m + log2f(l_run * f_self + l_o * f_other)) * LN2;
+      fence_before();
+      warp_arrive(smem_u32(o_free));
     }
   }
 
@@ -332,11 +416,10 @@ __global__ void __launch_bounds__(64 + 128 * NG, 1)
 // ld_qkv a multiple of 8 (checked by the caller).
 mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T,
                              int nq, int nkv, cudaStream_t st) {
-  constexpr int NG = 2;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attn_fwd_tc_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    attr = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr != cudaSuccess) return fail(MT_ERR_CUDA, "attention smem attribute: %s", cudaGetErrorString(attr));
   CUtensorMap tm;
@@ -344,10 +427,12 @@ mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t
                     static_cast<uint64_t>(ld), 64, 128));
   int32_t* err = device_error_word();
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
-  dim3 grid((T + BQ - 1) / BQ, nq, B);
+  const int64_t n_tiles = static_cast<int64_t>((T + BQ - 1) / BQ) * nq * B;
+  if (n_tiles >= (1ll << 31)) return fail(MT_ERR_INVALID_ARG, "attention: too many tiles");
+  const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
   const float scale_log2 = LOG2E / sqrtf(static_cast<float>(D));
-  attn_fwd_tc_kernel<NG><<<grid, 64 + 128 * NG, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, lse,
-                                                                  T, nq, nkv, scale_log2, err);
+  attn_fwd_tc_kernel<<<grid, FWD_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, lse, B, T,
+                                                            nq, nkv, scale_log2, err);
   MT_TRY(launch_check("attn_fwd_tc_kernel"));
   add_exec_flops(4.0 * B * nq * D * (0.5 * double(T) * double(T)));
   return MT_OK;
@@ -371,10 +456,14 @@ constexpr int HALF_TILE = 64 * D * 2;      // 16 KiB: 64 rows x 128 columns
 constexpr int HALF_ATOM = 64 * 64 * 2;     // 8 KiB: 64 rows of one 64-column atom
 
 // ------------------------------------------------------------ dK, dV
-// smem: K | V | Q0 dO0 | Q1 dO1 | PT0 DST0 | PT1 DST1 | lse/delta [2][2][64]
-constexpr int KV_OFF_K = 0, KV_OFF_V = TILE, KV_OFF_QO = 2 * TILE, KV_OFF_PD = 2 * TILE + 4 * HALF_TILE;
+// smem: K | V | Q0 dO0 | Q1 dO1 | Q2 dO2 | PT0 DST0 | PT1 DST1 | lse/delta [3][2][64]
+// Three Q / dO stages: the load of block it + 3 starts when the dV / dK MMAs of
+// block it are done, which leaves two blocks of work to cover its latency.
+constexpr int KV_QO_STAGES = 3;
+constexpr int KV_OFF_K = 0, KV_OFF_V = TILE, KV_OFF_QO = 2 * TILE;
+constexpr int KV_OFF_PD = KV_OFF_QO + KV_QO_STAGES * 2 * HALF_TILE;
 constexpr int KV_OFF_LD = KV_OFF_PD + 4 * ATOM;
-constexpr int KV_SMEM_TILES = KV_OFF_LD + 4 * 64 * 4;
+constexpr int KV_SMEM_TILES = KV_OFF_LD + KV_QO_STAGES * 128 * 4;
 constexpr int KV_SMEM_BYTES = KV_SMEM_TILES + 256 + 1024;
 constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;
 // Both backward kernels run two groups of four compute warps (warps 2-5 and 6-9),
@@ -391,18 +480,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   float* lsd = reinterpret_cast<float*>(smem + KV_OFF_LD);  // [stage][lse2 | delta][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KV_SMEM_TILES);
   uint64_t* kv_full = bars;       // 1
-  uint64_t* qo_full = bars + 1;   // 2
-  uint64_t* qo_empty = bars + 3;  // 2
-  uint64_t* sp_full = bars + 5;   // 2
-  uint64_t* pd_full = bars + 7;   // 2
-  uint64_t* mma_done = bars + 9;  // 2
-  uint64_t* fin = bars + 11;      // 1
-  uint64_t* l_bar = bars + 12;    // 1: lse/delta of a block written by the 128 compute threads
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* qo_full = bars + 1;   // 3
+  uint64_t* qo_empty = bars + 4;  // 3
+  uint64_t* l_full = bars + 7;    // 3: lse/delta of a stage written by the producer warp
+  uint64_t* sp_full = bars + 10;  // 2
+  uint64_t* pd_full = bars + 12;  // 2
+  uint64_t* mma_done = bars + 14; // 2
+  uint64_t* fin = bars + 16;      // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int kb = blockIdx.x;  // small key blocks have the most query blocks: first
-  const int c = blockIdx.y, b = blockIdx.z;
+  // key blocks vary slowest, so the launch order is small key blocks (the most query blocks) first
+  const int kb = blockIdx.z;
+  const int c = blockIdx.x, b = blockIdx.y;
   const int grp = nq / nkv;
   const int k0 = kb * 128;
   const int row0 = b * T;
@@ -416,14 +506,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(kv_full), 1);
     mbar_init(smem_u32(fin), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < KV_QO_STAGES; ++i) {
       mbar_init(smem_u32(&qo_full[i]), 1);
       mbar_init(smem_u32(&qo_empty[i]), 1);
+      mbar_init(smem_u32(&l_full[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sp_full[i]), 1);
-      mbar_init(smem_u32(&pd_full[i]), 256);
+      mbar_init(smem_u32(&pd_full[i]), 8);
       mbar_init(smem_u32(&mma_done[i]), 1);
     }
-    mbar_init(smem_u32(l_bar), 256);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -450,11 +542,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     __syncwarp();
     for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      if (!warp_wait(smem_u32(&qo_empty[st]), ((it >> 1) & 1) ^ 1, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+      const int st = it % KV_QO_STAGES;
+      const uint32_t par = static_cast<uint32_t>(it / KV_QO_STAGES) & 1u;
+      if (!warp_wait(smem_u32(&qo_empty[st]), par ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+      const int h = c * grp + it / per_head;
+      const int q0 = (qb0 + it % per_head) * 64;
       if (lane == 0) {
-        const int h = c * grp + it / per_head;
-        const int q0 = (qb0 + it % per_head) * 64;
         const uint32_t fb = smem_u32(&qo_full[st]);
         uint8_t* qt = smem + KV_OFF_QO + st * 2 * HALF_TILE;
         uint8_t* ot = qt + HALF_TILE;
@@ -464,7 +557,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tma_load_2d(smem_u32(ot), &tm_do64, fb, h * D, row0 + q0);
         tma_load_2d(smem_u32(ot + HALF_ATOM), &tm_do64, fb, h * D + 64, row0 + q0);
       }
-      __syncwarp();
+      // this block's log-sum-exp (log2 domain) and delta, shared by all key rows; rows past T give P = 0
+      const int64_t sb = (static_cast<int64_t>(b) * nq + h) * T;
+      float* l2 = lsd + st * 128;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int q = q0 + hh * 32 + lane;
+        l2[hh * 32 + lane] = q < T ? lse[sb + q] * LOG2E : INFINITY;
+        l2[64 + hh * 32 + lane] = q < T ? delta[sb + q] : 0.f;
+      }
+      warp_arrive(smem_u32(&l_full[st]));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -473,11 +575,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t k_base = smem_u32(smem + KV_OFF_K), v_base = smem_u32(smem + KV_OFF_V);
     bool ok = n_it == 0 || warp_wait(smem_u32(kv_full), 0, abort_flag, err, DEV_ERR_TIMEOUT_MMA);
     auto issue_sp = [&](int it) -> bool {
-      const int st = it & 1;
-      if (!warp_wait(smem_u32(&qo_full[st]), (it >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
+      const int st = it & 1, sq = it % KV_QO_STAGES;
+      if (!warp_wait(smem_u32(&qo_full[sq]), static_cast<uint32_t>(it / KV_QO_STAGES) & 1u, abort_flag, err,
+                     DEV_ERR_TIMEOUT_MMA))
+        return false;
       fence_after();
       if (lane == 0) {
-        const uint32_t q_base = smem_u32(smem + KV_OFF_QO + st * 2 * HALF_TILE);
+        const uint32_t q_base = smem_u32(smem + KV_OFF_QO + sq * 2 * HALF_TILE);
         const uint32_t o_base = q_base + HALF_TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -506,7 +610,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       fence_after();
       if (lane == 0) {
-        const uint32_t q_base = smem_u32(smem + KV_OFF_QO + st * 2 * HALF_TILE);
+        const int sq = it % KV_QO_STAGES;
+        const uint32_t q_base = smem_u32(smem + KV_OFF_QO + sq * 2 * HALF_TILE);
         const uint32_t o_base = q_base + HALF_TILE;
         const uint32_t pt = smem_u32(smem + KV_OFF_PD + st * 2 * ATOM);
         const uint32_t dst = pt + ATOM;
@@ -518,7 +623,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           umma_bf16(tmem + KV_COL_DK, smem_desc(dst + off_a, 16, 1024), smem_desc(q_base + kk * 2048, HALF_ATOM, 1024),
                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(smem_u32(&qo_empty[st]));
+        umma_commit(smem_u32(&qo_empty[sq]));
         umma_commit(smem_u32(&mma_done[st]));
       }
       __syncwarp();
@@ -530,29 +635,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int g = (warp - 2) >> 2;  // query columns [32 g, 32 g + 32) of each 64-column block
     const int qw = warp & 3;
     const int r = qw * 32 + lane;  // key row within the block
-    const int t = threadIdx.x - 64;  // 0..255 among the compute threads
     const int kv_row = k0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
-    uint32_t lph = 0;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      const int h = c * grp + it / per_head;
+      const int st = it & 1, sq = it % KV_QO_STAGES;
       const int q0 = (qb0 + it % per_head) * 64;
-      {  // this block's log-sum-exp (log2 domain) and delta, shared by all key rows
-        if (t < 128) {
-          const int q = q0 + (t & 63);
-          const int64_t sb = (static_cast<int64_t>(b) * nq + h) * T;
-          if (t < 64)
-            lsd[st * 128 + t] = q < T ? lse[sb + q] * LOG2E : INFINITY;
-          else
-            lsd[st * 128 + t] = q < T ? delta[sb + q] : 0.f;
-        }
-        if (!group_sync(smem_u32(l_bar), lph, abort_flag, err)) {
-          ok = false;
-          break;
-        }
+      if (!warp_wait(smem_u32(&l_full[sq]), static_cast<uint32_t>(it / KV_QO_STAGES) & 1u, abort_flag, err,
+                     DEV_ERR_TIMEOUT_EPILOGUE)) {
+        ok = false;
+        break;
       }
+      __syncwarp();  // lane 0's acquire of the producer's lse / delta stores covers the whole warp
       if (!warp_wait(smem_u32(&sp_full[st]), (it >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
         ok = false;
         break;
@@ -568,13 +662,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
       }
-      const float* L2 = lsd + st * 128 + g * 32;
+      const float* L2 = lsd + sq * 128 + g * 32;
       const float* Dl = L2 + 64;
       const int qc0 = q0 + g * 32;
       const bool diag = qc0 < k0 + 127;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        float p = exp2f(sv[e] * scale_log2 - L2[e]);
+        float p = ex2(fmaf(sv[e], scale_log2, -L2[e]));
         if (diag && kv_row > qc0 + e) p = 0.f;
         sv[e] = p;
         dv[e] = p * (dv[e] - Dl[e]);
@@ -604,7 +698,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       fence_proxy_async_smem();
       fence_before();
-      mbar_arrive(smem_u32(&pd_full[st]));
+      warp_arrive(smem_u32(&pd_full[st]));
     }
     if (ok && n_it > 0 && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
       fence_after();
@@ -643,8 +737,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }
 
 // ------------------------------------------------------------ dQ
-// smem: Q | dO | K0 V0 | K1 V1 | DS0 | DS1
-constexpr int DQ_OFF_Q = 0, DQ_OFF_O = TILE, DQ_OFF_KV = 2 * TILE, DQ_OFF_DS = 2 * TILE + 4 * HALF_TILE;
+// smem: Q | dO | K0 V0 | .. | K3 V3 | DS0 | DS1
+// Four K / V stages: the load of block j + 4 starts when the dQ MMAs of block j
+// are done, which leaves three blocks of work to cover its latency.
+constexpr int DQ_KV_STAGES = 4;
+constexpr int DQ_OFF_Q = 0, DQ_OFF_O = TILE, DQ_OFF_KV = 2 * TILE;
+constexpr int DQ_OFF_DS = DQ_OFF_KV + DQ_KV_STAGES * 2 * HALF_TILE;
 constexpr int DQ_SMEM_TILES = DQ_OFF_DS + 2 * ATOM;
 constexpr int DQ_SMEM_BYTES = DQ_SMEM_TILES + 256 + 1024;
 constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;
@@ -657,18 +755,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_SMEM_TILES);
-  uint64_t* q_full = bars;        // 1
-  uint64_t* kv_full = bars + 1;   // 2
-  uint64_t* kv_empty = bars + 3;  // 2
-  uint64_t* sp_full = bars + 5;   // 2
-  uint64_t* ds_full = bars + 7;   // 2
-  uint64_t* mma_done = bars + 9;  // 2
-  uint64_t* fin = bars + 11;      // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* q_full = bars;         // 1
+  uint64_t* kv_full = bars + 1;    // 4
+  uint64_t* kv_empty = bars + 5;   // 4
+  uint64_t* sp_full = bars + 9;    // 2
+  uint64_t* ds_full = bars + 11;   // 2
+  uint64_t* mma_done = bars + 13;  // 2
+  uint64_t* fin = bars + 15;       // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // query blocks vary slowest, so the launch order is the longest rows first
+  const int qb = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int c = (h * nkv) / nq;
   const int q0 = qb * 128;
   const int n_j = min((T + 63) / 64, (q0 + 128) / 64);
@@ -679,11 +778,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
     mbar_init(smem_u32(fin), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < DQ_KV_STAGES; ++i) {
       mbar_init(smem_u32(&kv_full[i]), 1);
       mbar_init(smem_u32(&kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sp_full[i]), 1);
-      mbar_init(smem_u32(&ds_full[i]), 256);
+      mbar_init(smem_u32(&ds_full[i]), 8);
       mbar_init(smem_u32(&mma_done[i]), 1);
     }
     *abort_flag = 0;
@@ -711,8 +812,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     __syncwarp();
     for (int j = 0; j < n_j; ++j) {
-      const int st = j & 1;
-      if (!warp_wait(smem_u32(&kv_empty[st]), ((j >> 1) & 1) ^ 1, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+      const int st = j % DQ_KV_STAGES;
+      const uint32_t par = static_cast<uint32_t>(j / DQ_KV_STAGES) & 1u;
+      if (!warp_wait(smem_u32(&kv_empty[st]), par ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
       if (lane == 0) {
         const uint32_t fb = smem_u32(&kv_full[st]);
         uint8_t* kt = smem + DQ_OFF_KV + st * 2 * HALF_TILE;
@@ -732,11 +834,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t q_base = smem_u32(smem + DQ_OFF_Q), o_base = smem_u32(smem + DQ_OFF_O);
     bool ok = warp_wait(smem_u32(q_full), 0, abort_flag, err, DEV_ERR_TIMEOUT_MMA);
     auto issue_sp = [&](int j) -> bool {
-      const int st = j & 1;
-      if (!warp_wait(smem_u32(&kv_full[st]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
+      const int st = j & 1, sk = j % DQ_KV_STAGES;
+      if (!warp_wait(smem_u32(&kv_full[sk]), static_cast<uint32_t>(j / DQ_KV_STAGES) & 1u, abort_flag, err,
+                     DEV_ERR_TIMEOUT_MMA))
+        return false;
       fence_after();
       if (lane == 0) {
-        const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + st * 2 * HALF_TILE);
+        const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + sk * 2 * HALF_TILE);
         const uint32_t v_base = k_base + HALF_TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -765,13 +869,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       fence_after();
       if (lane == 0) {
+        const int sk = j % DQ_KV_STAGES;
         const uint32_t ds = smem_u32(smem + DQ_OFF_DS + st * ATOM);
-        const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + st * 2 * HALF_TILE);
+        const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + sk * 2 * HALF_TILE);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
           umma_bf16(tmem + DQ_COL_DQ, smem_desc(ds + kk * 32, 16, 1024), smem_desc(k_base + kk * 2048, HALF_ATOM, 1024),
                     idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(smem_u32(&kv_empty[st]));
+        umma_commit(smem_u32(&kv_empty[sk]));
         umma_commit(smem_u32(&mma_done[st]));
       }
       __syncwarp();
@@ -809,7 +914,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const bool diag = k0 + 31 > q0;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        float p = exp2f(sv[e] * scale_log2 - lse2);
+        float p = ex2(fmaf(sv[e], scale_log2, -lse2));
         if (diag && k0 + e > q_row) p = 0.f;
         dv[e] = p * (dv[e] - dl);
       }
@@ -832,7 +937,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       fence_proxy_async_smem();
       fence_before();
-      mbar_arrive(smem_u32(&ds_full[st]));
+      warp_arrive(smem_u32(&ds_full[st]));
     }
     if (ok && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
       fence_after();
@@ -886,14 +991,16 @@ mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o,
   MT_TRY(tma_map_2d(&do64, d_o, o_cols, rows, static_cast<uint64_t>(ld_o), 64, 64));
   int32_t* err = device_error_word();
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
+  if (B > 65535 || (T + 127) / 128 > 65535 || nq > 65535)
+    return fail(MT_ERR_INVALID_ARG, "attention backward: B and T / 128 must be at most 65535");
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
   const float scale_log2 = LOG2E * scale;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(dqkv);
-  dim3 gq((T + 127) / 128, nq, B);
+  dim3 gq(nq, B, (T + 127) / 128);
   attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, T, nq, nkv,
                                                                 scale_log2, scale, err);
   MT_TRY(launch_check("attn_bwd_dq_tc_kernel"));
-  dim3 gk((T + 127) / 128, nkv, B);
+  dim3 gk(nkv, B, (T + 127) / 128);
   attn_bwd_dkv_tc_kernel<<<gk, BWD_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, T, nq, nkv,
                                                                  scale_log2, scale, err);
   MT_TRY(launch_check("attn_bwd_dkv_tc_kernel"));

@@ -55,9 +55,13 @@ struct EpiArgs {
   int M, N, K;
   int c_f32, accumulate;
   int raster;
-  // SwiGLU epilogue (2-SM kernel, both operands K-major): B holds [Wg; Wu] (N = 2F
-  // rows); a pair tile covers 128 features j, C[m, j] = silu(g) * u in bf16, and
-  // when gu is set g and u are also stored to gu[m, j] and gu[m, F + j].
+  // swiglu == 1, SwiGLU epilogue (2-SM kernel, both operands K-major): B holds
+  // [Wg; Wu] (N = 2F rows); a pair tile covers 128 features j, C[m, j] =
+  // silu(g) * u in bf16, and when gu is set g and u are also stored to gu[m, j]
+  // and gu[m, F + j].
+  // swiglu == 2, SwiGLU backward epilogue (any layout, N = F): the accumulator
+  // is dm[m, j]; g = gu[m, j] and u = gu[m, F + j] are read and replaced by
+  // dg = dm u silu'(g) and du = dm silu(g). C is not written.
   int swiglu, F;
   __nv_bfloat16* gu;
   int64_t ld_gu;
@@ -95,6 +99,15 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
 }
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with the MUFU ex2 and a fast divide
+// (relative error well below bf16 rounding; 2^x saturates to 0 / inf, giving
+// sigmoid 1 / 0 at the extremes).
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z));
+  return __fdividef(1.0f, 1.0f + e);
+}
 
 // Epilogue of one 32-column chunk of one output row.
 __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0, const uint32_t (&r)[32]) {
@@ -166,6 +179,54 @@ __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0
   }
 }
 
+// SwiGLU backward of 32 features of one row from the fp32 dm accumulators:
+// with s = sigmoid(g), dg = dm u s (1 + g (1 - s)) and du = dm g s, written over
+// g and u in place (each element is read and written by the same thread).
+__device__ __forceinline__ void store_swiglu_bwd(const EpiArgs& ep, int row, int f0, const uint32_t (&r)[32]) {
+  __nv_bfloat16* grow = ep.gu + static_cast<int64_t>(row) * ep.ld_gu;
+  if (f0 + 32 <= ep.F) {
+    uint4* gp = reinterpret_cast<uint4*>(grow + f0);
+    uint4* up = reinterpret_cast<uint4*>(grow + ep.F + f0);
+    // g and u are read once and written once: streaming loads / stores keep them from
+    // evicting the GEMM's operand tiles from L2; all eight loads are in flight together
+    uint4 ug[4], uu[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      ug[q] = __ldcs(gp + q);
+      uu[q] = __ldcs(up + q);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 og, ou;
+      const __nv_bfloat162* hg = reinterpret_cast<const __nv_bfloat162*>(&ug[q]);
+      const __nv_bfloat162* hu = reinterpret_cast<const __nv_bfloat162*>(&uu[q]);
+      __nv_bfloat162* dg = reinterpret_cast<__nv_bfloat162*>(&og);
+      __nv_bfloat162* du = reinterpret_cast<__nv_bfloat162*>(&ou);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 g = __bfloat1622float2(hg[j]), u = __bfloat1622float2(hu[j]);
+        const float d0 = __uint_as_float(r[q * 8 + 2 * j]), d1 = __uint_as_float(r[q * 8 + 2 * j + 1]);
+        const float s0 = sigmoid_fast(g.x), s1 = sigmoid_fast(g.y);
+        dg[j] = __floats2bfloat162_rn(d0 * u.x * s0 * (1.0f + g.x * (1.0f - s0)),
+                                      d1 * u.y * s1 * (1.0f + g.y * (1.0f - s1)));
+        du[j] = __floats2bfloat162_rn(d0 * g.x * s0, d1 * g.y * s1);
+      }
+      __stcs(gp + q, og);
+      __stcs(up + q, ou);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (f0 + j < ep.F) {
+        const float g = bf2f(grow[f0 + j]), u = bf2f(grow[ep.F + f0 + j]), d = __uint_as_float(r[j]);
+        const float sg = sigmoid_fast(g);
+        grow[f0 + j] = __float2bfloat16_rn(d * u * sg * (1.0f + g * (1.0f - sg)));
+        grow[ep.F + f0 + j] = __float2bfloat16_rn(d * g * sg);
+      }
+    }
+  }
+}
+
 // SwiGLU epilogue of 32 features of one row: m = silu(g) * u from the fp32
 // accumulators (g, u optionally stored too).
 __device__ __forceinline__ void store_swiglu(const EpiArgs& ep, int row, int f0, const uint32_t (&rg)[32],
@@ -174,7 +235,7 @@ __device__ __forceinline__ void store_swiglu(const EpiArgs& ep, int row, int f0,
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const float g = __uint_as_float(rg[j]), u = __uint_as_float(ru[j]);
-    m[j] = g / (1.0f + expf(-g)) * u;
+    m[j] = g * sigmoid_fast(g) * u;
   }
   __nv_bfloat16* mrow = static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc;
   __nv_bfloat16* grow = ep.gu ? ep.gu + static_cast<int64_t>(row) * ep.ld_gu : nullptr;
@@ -364,7 +425,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (col0 >= ep.N) break;  // uniform across the warp
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN + c * 32), r);
-        if (row < ep.M) store_chunk(ep, row, col0, r);
+        if (row < ep.M) {
+          if (ep.swiglu == 2)
+            store_swiglu_bwd(ep, row, col0, r);
+          else
+            store_chunk(ep, row, col0, r);
+        }
       }
       fence_before();
       mbar_arrive(smem_u32(&tempty[ab]));
@@ -496,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t rank = cluster_rank();
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int num_m = (ep.M + BM - 1) / BM;
-  const int num_n = ep.swiglu ? (ep.F + 127) / 128 : (ep.N + BN - 1) / BN;
+  const int num_n = ep.swiglu == 1 ? (ep.F + 127) / 128 : (ep.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (ep.K + BK - 1) / BK;
 
@@ -535,8 +601,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       const int m_own = mb * BM + static_cast<int>(rank) * 128;  // this CTA's A rows
       // this CTA's B rows (SwiGLU: the gate rows in the even CTA, the up rows in the odd one)
-      const int n_base0 = ep.swiglu ? nb * 128 : nb * BN;
-      const int n_base1 = ep.swiglu ? ep.F + nb * 128 : nb * BN + 128;
+      const int n_base0 = ep.swiglu == 1 ? nb * 128 : nb * BN;
+      const int n_base1 = ep.swiglu == 1 ? ep.F + nb * 128 : nb * BN + 128;
       const int n_own = rank == 0 ? n_base0 : n_base1;
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
@@ -632,7 +698,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
-      if (ep.swiglu) {
+      if (ep.swiglu == 1) {
         for (int c = 0; c < 4; ++c) {
           const int f0 = nb * 128 + c * 32;
           if (f0 >= ep.F) break;
@@ -647,7 +713,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (col0 >= ep.N) break;
           uint32_t r[32];
           tmem_ld32(tbase + static_cast<uint32_t>(c * 32), r);
-          if (row < ep.M) store_chunk(ep, row, col0, r);
+          if (row < ep.M) {
+            if (ep.swiglu == 2)
+              store_swiglu_bwd(ep, row, col0, r);
+            else
+              store_chunk(ep, row, col0, r);
+          }
         }
       }
       fence_before();
@@ -743,7 +814,7 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
                                     c2::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return fail(MT_ERR_CUDA, "gemm2 smem attribute: %s", cudaGetErrorString(attr_err));
-  const int num_n = ep.swiglu ? (ep.F + 127) / 128 : (ep.N + c2::BN - 1) / c2::BN;
+  const int num_n = ep.swiglu == 1 ? (ep.F + 127) / 128 : (ep.N + c2::BN - 1) / c2::BN;
   const int num_tiles = ((ep.M + c2::BM - 1) / c2::BM) * num_n;
   const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN, KA>());
   int32_t* err = device_error_word();
@@ -790,9 +861,13 @@ int pick_raster(int64_t M, int64_t N, int64_t K) {
 
 }  // namespace
 
-mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn, void* C,
-                      int64_t ldc, bool c_f32, bool accumulate, int64_t M, int64_t N, int64_t K,
-                      const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, cudaStream_t st) {
+namespace {
+
+// Tensor maps for the operands, then the kernel chosen by layout, timed by the
+// engine's observer. `ep` carries the epilogue; M, N, K come from it.
+mt_status gemm_dispatch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
+                        EpiArgs ep, cudaStream_t st) {
+  const int64_t M = ep.M, N = ep.N, K = ep.K;
   if (M == 0 || N == 0) return MT_OK;
   const bool two = use_2sm();
   const uint32_t b_rows = two ? 128 : BN;  // rows of a K-major B box
@@ -805,22 +880,7 @@ mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B
     MT_TRY(make_map(&tb, B, K, N, ldb, 64, b_rows));
   else
     MT_TRY(make_map(&tb, B, N, K, ldb, 64, 64));
-  EpiArgs ep;
-  ep.C = C;
-  ep.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
-  ep.res = reinterpret_cast<const __nv_bfloat16*>(residual);
-  ep.ldc = ldc;
-  ep.ldr = ldr;
-  ep.M = static_cast<int>(M);
-  ep.N = static_cast<int>(N);
-  ep.K = static_cast<int>(K);
-  ep.c_f32 = c_f32 ? 1 : 0;
-  ep.accumulate = accumulate ? 1 : 0;
   ep.raster = pick_raster(M, N, K);
-  ep.swiglu = 0;
-  ep.F = 0;
-  ep.gu = nullptr;
-  ep.ld_gu = 0;
   const double flops = 2.0 * double(M) * double(N) * double(K);
   GemmTimer* tm = current_gemm_timer();
   if (tm) tm->before(st);
@@ -847,6 +907,52 @@ mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B
   if (tm) tm->after(st, flops);
   add_exec_flops(flops);
   return s;
+}
+
+EpiArgs plain_epilogue(int64_t M, int64_t N, int64_t K) {
+  EpiArgs ep;
+  ep.C = nullptr;
+  ep.bias = nullptr;
+  ep.res = nullptr;
+  ep.ldc = 0;
+  ep.ldr = 0;
+  ep.M = static_cast<int>(M);
+  ep.N = static_cast<int>(N);
+  ep.K = static_cast<int>(K);
+  ep.c_f32 = 0;
+  ep.accumulate = 0;
+  ep.raster = 0;
+  ep.swiglu = 0;
+  ep.F = 0;
+  ep.gu = nullptr;
+  ep.ld_gu = 0;
+  return ep;
+}
+
+}  // namespace
+
+mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn, void* C,
+                      int64_t ldc, bool c_f32, bool accumulate, int64_t M, int64_t N, int64_t K,
+                      const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, cudaStream_t st) {
+  EpiArgs ep = plain_epilogue(M, N, K);
+  ep.C = C;
+  ep.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  ep.res = reinterpret_cast<const __nv_bfloat16*>(residual);
+  ep.ldc = ldc;
+  ep.ldr = ldr;
+  ep.c_f32 = c_f32 ? 1 : 0;
+  ep.accumulate = accumulate ? 1 : 0;
+  return gemm_dispatch(A, lda, a_mn, B, ldb, b_mn, ep, st);
+}
+
+mt_status gemm_swiglu_bwd_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
+                                 mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st) {
+  EpiArgs ep = plain_epilogue(M, F, K);
+  ep.swiglu = 2;
+  ep.F = static_cast<int>(F);
+  ep.gu = reinterpret_cast<__nv_bfloat16*>(gu);
+  ep.ld_gu = ld_gu;
+  return gemm_dispatch(A, lda, a_mn, B, ldb, b_mn, ep, st);
 }
 
 mt_status tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
@@ -924,4 +1030,17 @@ extern "C" mt_status mt_gemm_swiglu_bf16(const mt_bf16* A, int64_t lda, const mt
       F % 8 || (gu && ld_gu % 8))
     return fail(MT_ERR_ALIGNMENT, "gemm_swiglu: 16-byte alignment of pointers, rows and F");
   return gemm_swiglu_launch(A, lda, Wgu, ldw, m, ldm, gu, ld_gu, M, F, K, as_stream(stream));
+}
+
+extern "C" mt_status mt_gemm_swiglu_bwd_bf16(const mt_bf16* dY, int64_t ld_dy, const mt_bf16* Wd, int64_t ldw,
+                                             mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K,
+                                             void* stream) {
+  if (!dY || !Wd || !gu) return fail(MT_ERR_INVALID_ARG, "gemm_swiglu_bwd: dY, Wd and gu must not be NULL");
+  if (M < 0 || F <= 0 || K <= 0 || M >= (1ll << 31) || F >= (1ll << 30) || K >= (1ll << 31))
+    return fail(MT_ERR_INVALID_ARG, "gemm_swiglu_bwd: bad sizes");
+  if (ld_dy < K || ldw < F || ld_gu < 2 * F)
+    return fail(MT_ERR_INVALID_ARG, "gemm_swiglu_bwd: leading dimension smaller than the row it holds");
+  if (!aligned16(dY) || !aligned16(Wd) || !aligned16(gu) || ld_dy % 8 || ldw % 8 || ld_gu % 8 || F % 8)
+    return fail(MT_ERR_ALIGNMENT, "gemm_swiglu_bwd: 16-byte alignment of pointers, rows and F");
+  return gemm_swiglu_bwd_launch(dY, ld_dy, false, Wd, ldw, true, gu, ld_gu, M, F, K, as_stream(stream));
 }

@@ -25,8 +25,21 @@ mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, i
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
 mt_status rope_launch(mt_bf16*, int64_t, int, int, int, int, float, bool, cudaStream_t);
-mt_status swiglu_fwd_launch(const mt_bf16*, mt_bf16*, int64_t, int, cudaStream_t);
 mt_status swiglu_bwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, int64_t, int, cudaStream_t);
+
+// The SwiGLU backward runs in the epilogue of the dm GEMM unless
+// MT_SWIGLU_BWD=split selects the GEMM plus the stand-alone kernel (kept for
+// comparison measurements).
+bool swiglu_bwd_fused() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MT_SWIGLU_BWD");
+    v = (e && std::string(e) == "split") ? 0 : 1;
+  }
+  return v == 1;
+}
+
+mt_status swiglu_fwd_launch(const mt_bf16*, mt_bf16*, int64_t, int, cudaStream_t);
 mt_status colsum_launch(const mt_bf16*, const mt_bf16*, const float*, int64_t, int64_t, int64_t, float*, void*,
                         cudaStream_t);
 uint64_t colsum_ws_bytes(int64_t rows, int64_t cols);
@@ -199,11 +212,15 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
     // dWd (+)= dy^T m
     MT_TRY(gemm_launch(dyc, G.H, true, w.m, G.F, true, dw_dev + O.wd, G.F, true, acc, G.H, G.F, rows, nullptr, nullptr,
                        0, st));
-    // dm = dy Wd (into the m buffer)
-    MT_TRY(gemm_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.m, G.F, false, false, rows, G.F, G.H, nullptr,
-                       nullptr, 0, st));
-    // [dg|du] (in place over [g|u])
-    MT_TRY(swiglu_bwd_launch(w.m, w.gu, w.gu, rows, static_cast<int>(G.F), st));
+    if (swiglu_bwd_fused()) {
+      // dm = dy Wd, and in the same GEMM's epilogue [dg|du] in place over [g|u]
+      MT_TRY(gemm_swiglu_bwd_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.gu, 2 * G.F, rows, G.F, G.H, st));
+    } else {
+      // dm = dy Wd (into the m buffer), then [dg|du] in place over [g|u]
+      MT_TRY(gemm_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.m, G.F, false, false, rows, G.F, G.H, nullptr,
+                         nullptr, 0, st));
+      MT_TRY(swiglu_bwd_launch(w.m, w.gu, w.gu, rows, static_cast<int>(G.F), st));
+    }
     // dWgu (+)= dgu^T h2
     MT_TRY(gemm_launch(w.gu, 2 * G.F, true, h2c, G.H, true, dw_dev + O.wg, G.H, true, acc, 2 * G.F, G.H, rows, nullptr,
                        nullptr, 0, st));

@@ -88,6 +88,11 @@ mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B
                       void* C, int64_t ldc, bool c_f32, bool accumulate, int64_t M, int64_t N, int64_t K,
                       const mt_bf16* bias, const mt_bf16* residual, int64_t ldr, cudaStream_t st);
 
+// dm = A B (M x F) with the SwiGLU backward in the epilogue: gu holds [g | u]
+// (row stride ld_gu) on entry and [dg | du] on return; dm itself is not stored.
+mt_status gemm_swiglu_bwd_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
+                                 mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st);
+
 // GEMM launch observer (engine statistics): called around each GEMM launch.
 struct GemmTimer {
   virtual void before(cudaStream_t st) = 0;

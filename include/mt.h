@@ -156,6 +156,17 @@ mt_status mt_gemm_bf16(const mt_bf16* A, int64_t lda, int32_t a_mn_major,
 mt_status mt_gemm_swiglu_bf16(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m,
                               int64_t ldm, mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, void* stream);
 
+/* The MLP's input-gradient GEMM with the SwiGLU backward as its epilogue: dm =
+ * dY Wd (dY [M, K] K-major, Wd [K, F] row-major as stored in the layer record,
+ * K = hidden) is formed in fp32 and never stored; gu holds [g | u] (row r at
+ * gu + r * ld_gu, g in columns [0, F), u in [F, 2F)) on entry and
+ * [dg | du] = [dm u silu'(g) | dm silu(g)] (bf16) on return, in place. The
+ * SwiGLU derivative follows from the MLP's definition (Qwen2.5 block as read for
+ * MegaTrain's layer template). Pointers 16-byte aligned; ld_dy, ldw, ld_gu and
+ * F multiples of 8. MT_ERR_INVALID_ARG / MT_ERR_ALIGNMENT before any launch. */
+mt_status mt_gemm_swiglu_bwd_bf16(const mt_bf16* dY, int64_t ld_dy, const mt_bf16* Wd, int64_t ldw, mt_bf16* gu,
+                                  int64_t ld_gu, int64_t M, int64_t F, int64_t K, void* stream);
+
 /* RMSNorm forward over rows of H: y = x * rstd * g, rstd = 1/sqrt(mean x^2 + eps)
  * (fp32 [rows] out). */
 mt_status mt_rmsnorm_fwd(const mt_bf16* x, const mt_bf16* g, mt_bf16* y, float* rstd,

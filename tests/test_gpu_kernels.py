@@ -103,6 +103,34 @@ def test_gemm_with_swiglu_epilogue(M, F, K):
     assert torch.equal(m.view(torch.int16), m2.view(torch.int16))
 
 
+@pytest.mark.parametrize("M,F,K", [(256, 688, 256), (200, 1000, 136), (8192, 18944, 3584)])
+def test_gemm_with_swiglu_backward_epilogue(M, F, K):
+    """dm = dY Wd with [g|u] replaced by [dg|du] in the epilogue, against the
+    oracle's SwiGLU backward on the float64 product."""
+    import torch
+    dY = _bits(11, 1, M * K, 1.0).reshape(M, K)
+    Wd = _bits(11, 2, K * F, 0.05).reshape(K, F)  # [hidden, F] as stored in the layer record
+    gu = _bits(11, 3, M * 2 * F, 2.0).reshape(M, 2 * F)
+    gud = H.dev_bf16(gu)
+    L.mt_gemm_swiglu_bwd_bf16(H.dev_bf16(dY), K, H.dev_bf16(Wd), F, gud, 2 * F, M, F, K)
+    torch.cuda.synchronize()
+    _check_dev_error()
+    rows = np.arange(M) if M <= 256 else np.random.default_rng(1).choice(M, 96, replace=False)
+    dm = H.bits_to_f64(dY)[rows] @ H.bits_to_f64(Wd)
+    g64, u64 = H.bits_to_f64(gu[rows, :F]), H.bits_to_f64(gu[rows, F:])
+    dg, du = O.swiglu_bwd(dm, g64, u64)
+    got = H.host_f64(gud)[rows]
+    assert H.rel(got[:, :F], dg) < 1e-2
+    assert H.rel(got[:, F:], du) < 1e-2
+    # the same GEMM plus the stand-alone SwiGLU backward kernel agrees (dm rounded to bf16 there)
+    dmd = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+    L.mt_gemm_bf16(H.dev_bf16(dY), K, 0, H.dev_bf16(Wd), F, 1, dmd, F, 0, 0, M, F, K, None, None, 0)
+    dgu = H.empty_bf16(M, 2 * F)
+    L.mt_swiglu_bwd(dmd, H.dev_bf16(gu), dgu, M, F)
+    torch.cuda.synchronize()
+    assert H.rel(got, H.host_f64(dgu)[rows]) < 1e-2
+
+
 # ------------------------------------------------------------------ RMSNorm
 @pytest.mark.parametrize("rows,Hd", [(256, 256), (1000, 3584), (37, 5120)])
 def test_rmsnorm_forward_and_backward(rows, Hd):
@@ -195,6 +223,8 @@ ATTN_CASES = [
     (2, 64, 2, 1, 128),
     (2, 1024, 28, 4, 128),  # the 7B heads over 8 key blocks (online-softmax rescaling)
     (2, 700, 8, 2, 128),    # ragged last query block that reaches into the next sequence and past the end
+    (3, 1, 7, 1, 128),      # one token: the upper key half of the only block is masked for every row
+    (3, 37, 5, 5, 128),     # shorter than one key half
 ]
 
 

@@ -6,7 +6,7 @@
 // tiles, longest rows first, so the next tile's Q load and first two S MMAs
 // overlap the current tile's output epilogue.
 //   warp 0     TMA: lane 0 loads Q per tile and K_j, lane 1 V_j (128 key
-//              rows each), each into its own two-stage ring: a K stage is
+//              rows each), each into its own three-stage ring: a K stage is
 //              free once S_j is done, a V stage once O += P_j V_j is;
 //   warp 1     TMEM allocation and the MMA issuer: S_{j+1} = Q K_{j+1}^T is
 //              issued before O += P_j V_j so the tensor cores work while the
@@ -18,6 +18,11 @@
 //              inside the CTA), so the groups never synchronise inside the
 //              key loop; the two partial results meet once per tile:
 //              O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)).
+// P never touches shared memory: each thread writes its row of P_g (bf16
+// pairs) over the first 32 columns of its own half of the S buffer it just
+// read, and O_g += P_g V_g takes its A operand from tensor memory. The
+// tensor core runs one CTA's MMAs in issue order, so S_{j+2}, issued after
+// O += P_j V_j, cannot overwrite P_j before that MMA has read it.
 // Scores are handled in the log2 domain. TMEM: two S buffers (128 columns
 // each), O_0 and O_1 (128 columns each). O_g is rescaled only when its row
 // maximum grows by more than 8 (a factor 256 in the exponent); otherwise the
@@ -37,9 +42,10 @@ using namespace tc;
 constexpr int D = 128, BQ = 128, BKV = 128;
 constexpr int TILE = BQ * D * 2;  // 32 KiB: a 128 x 128 bf16 tile (two 64-column swizzle atoms)
 constexpr int ATOM = 128 * 64 * 2;  // 16 KiB
-// shared memory: Q | K0 V0 | K1 V1 | P0 | P1
-constexpr int OFF_Q = 0, OFF_KV = TILE, OFF_P = 5 * TILE;
-constexpr int SMEM_TILES = 7 * TILE;
+// shared memory: Q | K0 V0 | K1 V1 | K2 V2 | row exchange [3][128] floats
+constexpr int KV_STAGES = 3;
+constexpr int OFF_Q = 0, OFF_KV = TILE, OFF_X = TILE + KV_STAGES * 2 * TILE;
+constexpr int SMEM_TILES = OFF_X + 3 * 128 * 4;
 constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;  // tiles, barriers, alignment
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_O = 256;  // S_s at 128 s, O_g at 256 + 128 g
@@ -77,6 +83,28 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Each thread of the warp writes 16 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D (+)= A B with A (M = 128 rows in the lanes, 16 bf16 of K packed in pairs
+// along 8 columns) read from tensor memory and B from shared memory.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // Tile t of the persistent walk: query blocks from the last (longest rows)
 // down, then query head, then sequence.
 struct FwdTile {
@@ -96,19 +124,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
   uint64_t* q_full = bars;        // 1: Q of the tile loaded
   uint64_t* q_empty = bars + 1;   // 1: the tile's S MMAs (the readers of Q) are done
-  uint64_t* k_full = bars + 2;    // 2
-  uint64_t* k_empty = bars + 4;   // 2
-  uint64_t* v_full = bars + 6;    // 2
-  uint64_t* v_empty = bars + 8;   // 2
-  uint64_t* s_full = bars + 10;   // 2
-  uint64_t* p_full = bars + 12;   // [group][buffer]: 4, one arrival per warp of the group
-  uint64_t* o_done = bars + 16;   // [group][buffer]: 4
-  uint64_t* o_free = bars + 20;   // 1: the tile's O accumulators have been read (8 warps)
-  uint64_t* x_bar = bars + 21;    // 1: row exchange between the groups (8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* k_full = bars + 2;    // 3
+  uint64_t* k_empty = bars + 5;   // 3
+  uint64_t* v_full = bars + 8;    // 3
+  uint64_t* v_empty = bars + 11;  // 3
+  uint64_t* s_full = bars + 14;   // 2
+  uint64_t* p_full = bars + 16;   // [group][buffer]: 4, one arrival per warp of the group
+  uint64_t* o_done = bars + 20;   // [group][buffer]: 4
+  uint64_t* o_free = bars + 24;   // 1: the tile's O accumulators have been read (8 warps)
+  uint64_t* x_bar = bars + 25;    // 1: row exchange between the groups (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // the groups' row maxima and sums meet in P buffer 0, which is idle by then: [m | l][group][128 rows]
-  float* xch = reinterpret_cast<float*>(smem + OFF_P);
+  float* xch = reinterpret_cast<float*>(smem + OFF_X);  // [3][128]: group 1's (m, l), then group 0's (f0, f1, 1/l)
 
   const int n_qb = (T + BQ - 1) / BQ;
   const int n_tiles = n_qb * nq * B;
@@ -117,13 +144,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
     mbar_init(smem_u32(q_empty), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < KV_STAGES; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
-      mbar_init(smem_u32(&s_full[i]), 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&s_full[i]), 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&p_full[i]), 4);
       mbar_init(smem_u32(&o_done[i]), 1);
@@ -168,8 +195,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         uint64_t* empty = lane == 0 ? k_empty : v_empty;
         const int off = lane == 0 ? 0 : TILE;
         for (int j = 0; j < n_kv; ++j, ++it) {
-          const int s = it & 1;
-          if (!mbar_wait(smem_u32(&empty[s]), ((it >> 1) & 1u) ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+          const int s = it % KV_STAGES;
+          if (!mbar_wait(smem_u32(&empty[s]), ((it / KV_STAGES) & 1u) ^ 1u, abort_flag, err,
+                         DEV_ERR_TIMEOUT_PRODUCER)) {
             ok = false;
             break;
           }
@@ -189,11 +217,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);     // O_g += P_g V_g: V is MN-major (d contiguous)
     const uint32_t q_base = smem_u32(smem + OFF_Q);
     auto issue_s = [&](uint32_t i) -> bool {
-      const int s = i & 1;
-      if (!warp_wait(smem_u32(&k_full[s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
+      const int s = i & 1, sk = i % KV_STAGES;
+      if (!warp_wait(smem_u32(&k_full[sk]), (i / KV_STAGES) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) return false;
       fence_after();
       if (lane == 0) {
-        const uint32_t k_base = smem_u32(smem + OFF_KV + s * 2 * TILE);
+        const uint32_t k_base = smem_u32(smem + OFF_KV + sk * 2 * TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk >> 2) * ATOM + (kk & 3) * 32);
@@ -201,7 +229,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(smem_u32(&s_full[s]));
-        umma_commit(smem_u32(&k_empty[s]));
+        umma_commit(smem_u32(&k_empty[sk]));
       }
       __syncwarp();
       return true;
@@ -229,9 +257,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           ok = false;
           break;
         }
-        const uint32_t p_base = smem_u32(smem + OFF_P + s * TILE);
-        const uint32_t v_base = smem_u32(smem + OFF_KV + s * 2 * TILE + TILE);
-        if (!warp_wait(smem_u32(&v_full[s]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+        const int sv = i % KV_STAGES;
+        const uint32_t v_base = smem_u32(smem + OFF_KV + sv * 2 * TILE + TILE);
+        if (!warp_wait(smem_u32(&v_full[sv]), (i / KV_STAGES) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
@@ -242,13 +270,15 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           }
           fence_after();
           if (lane == 0) {
+            // P_g sits in the first 32 columns of group g's half of S buffer s
+            const uint32_t p_tmem = tmem + COL_S0 + s * BKV + g * 64;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              umma_bf16(tmem + COL_O + g * D, smem_desc(p_base + g * ATOM + kk * 32, 16, 1024),
-                        smem_desc(v_base + (g * 4 + kk) * 2048, ATOM, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16_tmem_a(tmem + COL_O + g * D, p_tmem + kk * 8, smem_desc(v_base + (g * 4 + kk) * 2048, ATOM, 1024),
+                               idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(smem_u32(&o_done[g * 2 + s]));
-            if (g == 1) umma_commit(smem_u32(&v_empty[s]));
+            if (g == 1) umma_commit(smem_u32(&v_empty[sv]));
           }
           __syncwarp();
         }
@@ -323,32 +353,20 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           l_run *= alpha;
           m_run = m_new;
         }
-        // P V of block i - 2 must be done reading this group's half of P buffer s
-        if (i >= 2 && !warp_wait(smem_u32(&o_done[g * 2 + s]), ((i - 2) >> 1) & 1u, abort_flag, err,
-                                 DEV_ERR_TIMEOUT_EPILOGUE)) {
-          ok = false;
-          break;
-        }
+        // P over the S values just read (its MMA reader of two blocks ago finished before S_i was
+        // written: the tensor core runs the CTA's MMAs in order and s_full covers all earlier ones)
         const float mb = m_run == -INFINITY ? 0.f : m_run;  // a fully masked row half gives P = 0
-        uint8_t* prow = smem + OFF_P + s * TILE + g * ATOM + r * 128;
         float lsum = 0.f;
+        uint32_t pk[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunks of 8 columns
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = ex2(fmaf(sv[ch * 8 + e], scale_log2, -mb));
-            lsum += p[e];
-          }
-          uint4 wv;
-          wv.x = pack_bf16(p[0], p[1]);
-          wv.y = pack_bf16(p[2], p[3]);
-          wv.z = pack_bf16(p[4], p[5]);
-          wv.w = pack_bf16(p[6], p[7]);
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = wv;
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2(fmaf(sv[2 * e], scale_log2, -mb));
+          const float p1 = ex2(fmaf(sv[2 * e + 1], scale_log2, -mb));
+          lsum += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
         }
+        tmem_st32(tmem + lane_base + COL_S0 + s * BKV + g * 64, pk);
         l_run += lsum;
-        fence_proxy_async_smem();
         fence_before();
         warp_arrive(smem_u32(&p_full[g * 2 + s]));
       }
@@ -363,15 +381,31 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         break;
       }
       fence_after();
-      xch[g * 128 + r] = m_run;
-      xch[256 + g * 128 + r] = l_run;
+      // group 1 hands its (m, l) to group 0, which forms the combination and hands back (f0, f1, 1/l)
+      if (g == 1) {
+        xch[r] = m_run;
+        xch[128 + r] = l_run;
+      }
       if (!warps_sync(smem_u32(x_bar), xph, abort_flag, err)) break;
-      const float m_o = xch[(g ^ 1) * 128 + r], l_o = xch[256 + (g ^ 1) * 128 + r];
-      if (!warps_sync(smem_u32(x_bar), xph, abort_flag, err)) break;  // both read before P is written again
-      const float m = fmaxf(m_run, m_o);
-      const float f_self = ex2(m_run - m), f_other = ex2(m_o - m);
-      const float inv = 1.f / (l_run * f_self + l_o * f_other);
-      const float f0 = g == 0 ? f_self : f_other, f1 = g == 0 ? f_other : f_self;
+      float f0, f1, inv;
+      if (g == 0) {
+        const float m1 = xch[r], l1 = xch[128 + r];
+        const float m = fmaxf(m_run, m1);
+        f0 = ex2(m_run - m);
+        f1 = ex2(m1 - m);
+        const float l_tot = l_run * f0 + l1 * f1;
+        inv = 1.f / l_tot;
+        xch[r] = f0;
+        xch[128 + r] = f1;
+        xch[256 + r] = inv;
+        if (q_row < T) lse[(static_cast<int64_t>(w.b) * nq + w.h) * T + q_row] = (m + log2f(l_tot)) * LN2;
+      }
+      if (!warps_sync(smem_u32(x_bar), xph, abort_flag, err)) break;
+      if (g == 1) {
+        f0 = xch[r];
+        f1 = xch[128 + r];
+        inv = xch[256 + r];
+      }
       __nv_bfloat16* orow = o + (static_cast<int64_t>(row0) + q_row) * ld_o + static_cast<int64_t>(w.h) * D;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {  // this group writes output columns [64 g, 64 g + 64)
@@ -395,8 +429,6 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           }
         }
       }
-      if (q_row < T && g == 0)
-        lse[(static_cast<int64_t>(w.b) * nq + w.h) * T + q_row] = (m + log2f(l_run * f_self + l_o * f_other)) * LN2;
       fence_before();
       warp_arrive(smem_u32(o_free));
     }
@@ -456,13 +488,17 @@ constexpr int HALF_TILE = 64 * D * 2;      // 16 KiB: 64 rows x 128 columns
 constexpr int HALF_ATOM = 64 * 64 * 2;     // 8 KiB: 64 rows of one 64-column atom
 
 // ------------------------------------------------------------ dK, dV
-// smem: K | V | Q0 dO0 | Q1 dO1 | Q2 dO2 | PT0 DST0 | PT1 DST1 | lse/delta [3][2][64]
-// Three Q / dO stages: the load of block it + 3 starts when the dV / dK MMAs of
-// block it are done, which leaves two blocks of work to cover its latency.
-constexpr int KV_QO_STAGES = 3;
+// smem: K | V | Q0 dO0 | .. | Q3 dO3 | lse/delta [4][2][64]
+// Four Q / dO stages: the load of block it + 4 starts when the dV / dK MMAs of
+// block it are done, which leaves three blocks of work to cover its latency.
+// P^T and dS^T never touch shared memory: each thread writes its key row of
+// them (bf16 pairs) over the first 16 columns of its group's half of the S^T
+// and dP^T buffers it just read, and dV += P^T dO, dK += dS^T Q take their A
+// operand from tensor memory (the tensor core runs the CTA's MMAs in issue
+// order, so S^T / dP^T of block it + 2 cannot overwrite them before they are read).
+constexpr int KV_QO_STAGES = 4;
 constexpr int KV_OFF_K = 0, KV_OFF_V = TILE, KV_OFF_QO = 2 * TILE;
-constexpr int KV_OFF_PD = KV_OFF_QO + KV_QO_STAGES * 2 * HALF_TILE;
-constexpr int KV_OFF_LD = KV_OFF_PD + 4 * ATOM;
+constexpr int KV_OFF_LD = KV_OFF_QO + KV_QO_STAGES * 2 * HALF_TILE;
 constexpr int KV_SMEM_TILES = KV_OFF_LD + KV_QO_STAGES * 128 * 4;
 constexpr int KV_SMEM_BYTES = KV_SMEM_TILES + 256 + 1024;
 constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;
@@ -480,14 +516,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   float* lsd = reinterpret_cast<float*>(smem + KV_OFF_LD);  // [stage][lse2 | delta][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KV_SMEM_TILES);
   uint64_t* kv_full = bars;       // 1
-  uint64_t* qo_full = bars + 1;   // 3
-  uint64_t* qo_empty = bars + 4;  // 3
-  uint64_t* l_full = bars + 7;    // 3: lse/delta of a stage written by the producer warp
-  uint64_t* sp_full = bars + 10;  // 2
-  uint64_t* pd_full = bars + 12;  // 2
-  uint64_t* mma_done = bars + 14; // 2
-  uint64_t* fin = bars + 16;      // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* qo_full = bars + 1;   // 4
+  uint64_t* qo_empty = bars + 5;  // 4
+  uint64_t* l_full = bars + 9;    // 4: lse/delta of a stage written by the producer warp
+  uint64_t* sp_full = bars + 13;  // 2
+  uint64_t* pd_full = bars + 15;  // 2
+  uint64_t* mma_done = bars + 17; // 2
+  uint64_t* fin = bars + 19;      // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // key blocks vary slowest, so the launch order is small key blocks (the most query blocks) first
@@ -613,15 +649,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const int sq = it % KV_QO_STAGES;
         const uint32_t q_base = smem_u32(smem + KV_OFF_QO + sq * 2 * HALF_TILE);
         const uint32_t o_base = q_base + HALF_TILE;
-        const uint32_t pt = smem_u32(smem + KV_OFF_PD + st * 2 * ATOM);
-        const uint32_t dst = pt + ATOM;
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk) {
-          const uint32_t off_a = static_cast<uint32_t>(kk * 32);
-          umma_bf16(tmem + KV_COL_DV, smem_desc(pt + off_a, 16, 1024), smem_desc(o_base + kk * 2048, HALF_ATOM, 1024),
-                    idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + KV_COL_DK, smem_desc(dst + off_a, 16, 1024), smem_desc(q_base + kk * 2048, HALF_ATOM, 1024),
-                    idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+          // query columns [16 kk, 16 kk + 16): group kk / 2's packed columns, second half at + 8
+          const uint32_t a_col = static_cast<uint32_t>(st * 64 + (kk >> 1) * 32 + (kk & 1) * 8);
+          umma_bf16_tmem_a(tmem + KV_COL_DV, tmem + KV_COL_ST + a_col, smem_desc(o_base + kk * 2048, HALF_ATOM, 1024),
+                           idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + KV_COL_DK, tmem + KV_COL_DPT + a_col, smem_desc(q_base + kk * 2048, HALF_ATOM, 1024),
+                           idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(smem_u32(&qo_empty[sq]));
         umma_commit(smem_u32(&mma_done[st]));
@@ -673,30 +708,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         sv[e] = p;
         dv[e] = p * (dv[e] - Dl[e]);
       }
-      if (it >= 2) {  // the dV/dK MMAs of it-2 must be done reading this P^T / dS^T buffer
-        if (!warp_wait(smem_u32(&mma_done[st]), ((it - 2) >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
-          ok = false;
-          break;
-        }
-      }
-      uint8_t* prow = smem + KV_OFF_PD + st * 2 * ATOM + r * 128;
+      {  // P^T and dS^T over the S^T / dP^T values just read
+        uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c16 = g * 4 + ch;
-        uint4 wp, wd;
-        wp.x = pack_bf16(sv[ch * 8 + 0], sv[ch * 8 + 1]);
-        wp.y = pack_bf16(sv[ch * 8 + 2], sv[ch * 8 + 3]);
-        wp.z = pack_bf16(sv[ch * 8 + 4], sv[ch * 8 + 5]);
-        wp.w = pack_bf16(sv[ch * 8 + 6], sv[ch * 8 + 7]);
-        wd.x = pack_bf16(dv[ch * 8 + 0], dv[ch * 8 + 1]);
-        wd.y = pack_bf16(dv[ch * 8 + 2], dv[ch * 8 + 3]);
-        wd.z = pack_bf16(dv[ch * 8 + 4], dv[ch * 8 + 5]);
-        wd.w = pack_bf16(dv[ch * 8 + 6], dv[ch * 8 + 7]);
-        const int sw = (c16 ^ (r & 7)) << 4;
-        *reinterpret_cast<uint4*>(prow + sw) = wp;
-        *reinterpret_cast<uint4*>(prow + ATOM + sw) = wd;
+        for (int e = 0; e < 16; ++e) {
+          pp[e] = pack_bf16(sv[2 * e], sv[2 * e + 1]);
+          pd[e] = pack_bf16(dv[2 * e], dv[2 * e + 1]);
+        }
+        tmem_st16(tmem + lane_base + KV_COL_ST + st * 64 + g * 32, pp);
+        tmem_st16(tmem + lane_base + KV_COL_DPT + st * 64 + g * 32, pd);
       }
-      fence_proxy_async_smem();
       fence_before();
       warp_arrive(smem_u32(&pd_full[st]));
     }
@@ -737,13 +758,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }
 
 // ------------------------------------------------------------ dQ
-// smem: Q | dO | K0 V0 | .. | K3 V3 | DS0 | DS1
-// Four K / V stages: the load of block j + 4 starts when the dQ MMAs of block j
-// are done, which leaves three blocks of work to cover its latency.
-constexpr int DQ_KV_STAGES = 4;
+// smem: Q | dO | K0 V0 | .. | K4 V4
+// Five K / V stages: the load of block j + 5 starts when the dQ MMAs of block j
+// are done, which leaves four blocks of work to cover its latency. dS never
+// touches shared memory: each thread writes its row of it (bf16 pairs) over
+// the first 16 columns of its group's half of the S buffer it just read, and
+// dQ += dS K takes its A operand from tensor memory.
+constexpr int DQ_KV_STAGES = 5;
 constexpr int DQ_OFF_Q = 0, DQ_OFF_O = TILE, DQ_OFF_KV = 2 * TILE;
-constexpr int DQ_OFF_DS = DQ_OFF_KV + DQ_KV_STAGES * 2 * HALF_TILE;
-constexpr int DQ_SMEM_TILES = DQ_OFF_DS + 2 * ATOM;
+constexpr int DQ_SMEM_TILES = DQ_OFF_KV + DQ_KV_STAGES * 2 * HALF_TILE;
 constexpr int DQ_SMEM_BYTES = DQ_SMEM_TILES + 256 + 1024;
 constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;
 
@@ -756,13 +779,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_SMEM_TILES);
   uint64_t* q_full = bars;         // 1
-  uint64_t* kv_full = bars + 1;    // 4
-  uint64_t* kv_empty = bars + 5;   // 4
-  uint64_t* sp_full = bars + 9;    // 2
-  uint64_t* ds_full = bars + 11;   // 2
-  uint64_t* mma_done = bars + 13;  // 2
-  uint64_t* fin = bars + 15;       // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kv_full = bars + 1;    // 5
+  uint64_t* kv_empty = bars + 6;   // 5
+  uint64_t* sp_full = bars + 11;   // 2
+  uint64_t* ds_full = bars + 13;   // 2
+  uint64_t* mma_done = bars + 15;  // 2
+  uint64_t* fin = bars + 17;       // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // query blocks vary slowest, so the launch order is the longest rows first
@@ -870,12 +893,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       fence_after();
       if (lane == 0) {
         const int sk = j % DQ_KV_STAGES;
-        const uint32_t ds = smem_u32(smem + DQ_OFF_DS + st * ATOM);
         const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + sk * 2 * HALF_TILE);
 #pragma unroll
-        for (int kk = 0; kk < 64 / 16; ++kk)
-          umma_bf16(tmem + DQ_COL_DQ, smem_desc(ds + kk * 32, 16, 1024), smem_desc(k_base + kk * 2048, HALF_ATOM, 1024),
-                    idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 64 / 16; ++kk) {
+          // key columns [16 kk, 16 kk + 16): group kk / 2's packed columns, second half at + 8
+          const uint32_t a_col = static_cast<uint32_t>(st * 64 + (kk >> 1) * 32 + (kk & 1) * 8);
+          umma_bf16_tmem_a(tmem + DQ_COL_DQ, tmem + DQ_COL_S + a_col, smem_desc(k_base + kk * 2048, HALF_ATOM, 1024),
+                           idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         umma_commit(smem_u32(&kv_empty[sk]));
         umma_commit(smem_u32(&mma_done[st]));
       }
@@ -918,24 +943,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (diag && k0 + e > q_row) p = 0.f;
         dv[e] = p * (dv[e] - dl);
       }
-      if (j >= 2) {
-        if (!warp_wait(smem_u32(&mma_done[st]), ((j - 2) >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
-          ok = false;
-          break;
-        }
-      }
-      uint8_t* drow = smem + DQ_OFF_DS + st * ATOM + r * 128;
+      {  // dS over the S values just read
+        uint32_t pd[16];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c16 = g * 4 + ch;
-        uint4 w;
-        w.x = pack_bf16(dv[ch * 8 + 0], dv[ch * 8 + 1]);
-        w.y = pack_bf16(dv[ch * 8 + 2], dv[ch * 8 + 3]);
-        w.z = pack_bf16(dv[ch * 8 + 4], dv[ch * 8 + 5]);
-        w.w = pack_bf16(dv[ch * 8 + 6], dv[ch * 8 + 7]);
-        *reinterpret_cast<uint4*>(drow + ((c16 ^ (r & 7)) << 4)) = w;
+        for (int e = 0; e < 16; ++e) pd[e] = pack_bf16(dv[2 * e], dv[2 * e + 1]);
+        tmem_st16(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, pd);
       }
-      fence_proxy_async_smem();
       fence_before();
       warp_arrive(smem_u32(&ds_full[st]));
     }

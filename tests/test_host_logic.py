@@ -128,6 +128,18 @@ def test_invalid_arguments_are_rejected_without_a_gpu():
     assert e.value.name == "MT_ERR_UNSUPPORTED"
     opts = L.make_opts(ckpt_interval=0)
     assert L.mt_engine_workspace_bytes(L.make_cfg(**TINY), 2, 1, 8, opts) == 0
+    with pytest.raises(L.MTError) as e:  # the hooked step checks its arguments before any work
+        L.mt_stream_step_hooked(None, None, None, None, None, None)
+    assert e.value.name == "MT_ERR_INVALID_ARG"
+    with pytest.raises(L.MTError) as e:
+        L.mt_gemm_swiglu_bwd_bf16(16, 8, 16, 8, 16, 8, 8, 8, 8)  # ld_gu < 2 F
+    assert e.value.name == "MT_ERR_INVALID_ARG"
+    with pytest.raises(L.MTError) as e:
+        L.mt_gemm_swiglu_bwd_bf16(16, 8, 16, 8, 16, 12, 8, 6, 8)  # F not a multiple of 8
+    assert e.value.name == "MT_ERR_ALIGNMENT"
+    with pytest.raises(L.MTError) as e:
+        L.mt_head_loss_fwd_bwd(16, 16, 16, 16, 8, 12, 16, 1e-6, 8, 16, 16, 16, 16, 16, 1 << 20)  # H % 8
+    assert e.value.name == "MT_ERR_INVALID_ARG"
 
 
 def test_tflops_formula_reproduces_table7_long_context_rows():

@@ -521,9 +521,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* l_full = bars + 9;    // 4: lse/delta of a stage written by the producer warp
   uint64_t* sp_full = bars + 13;  // 2
   uint64_t* pd_full = bars + 15;  // 2
-  uint64_t* mma_done = bars + 17; // 2
-  uint64_t* fin = bars + 19;      // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* fin = bars + 17;      // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // key blocks vary slowest, so the launch order is small key blocks (the most query blocks) first
@@ -550,7 +549,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sp_full[i]), 1);
       mbar_init(smem_u32(&pd_full[i]), 8);
-      mbar_init(smem_u32(&mma_done[i]), 1);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -659,7 +657,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                            idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(smem_u32(&qo_empty[sq]));
-        umma_commit(smem_u32(&mma_done[st]));
       }
       __syncwarp();
     }
@@ -783,9 +780,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* kv_empty = bars + 6;   // 5
   uint64_t* sp_full = bars + 11;   // 2
   uint64_t* ds_full = bars + 13;   // 2
-  uint64_t* mma_done = bars + 15;  // 2
-  uint64_t* fin = bars + 17;       // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* fin = bars + 15;       // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // query blocks vary slowest, so the launch order is the longest rows first
@@ -808,7 +804,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sp_full[i]), 1);
       mbar_init(smem_u32(&ds_full[i]), 8);
-      mbar_init(smem_u32(&mma_done[i]), 1);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -902,7 +897,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                            idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(smem_u32(&kv_empty[sk]));
-        umma_commit(smem_u32(&mma_done[st]));
       }
       __syncwarp();
     }

@@ -39,9 +39,11 @@ struct Use {
 };
 std::vector<Use> build_uses(int L, int K);
 void plan_slots(const std::vector<Use>& u, int R, std::vector<int>& slot, std::vector<int>& load);
+mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
+                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep);
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done);
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd);
 }  // namespace mt
 
 using namespace mt;
@@ -420,12 +422,17 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       status = cuda_check(cudaStreamWaitEvent(e->cs, e->ready[e->load_of_use[i]], 0), "wait weights");
       if (status != MT_OK) break;
     }
+    // the backward of a layer that directly follows its own forward (the top layer) finds
+    // the forward's internals still in the layer workspace and skips their recompute
+    const bool fwd_then_bwd = i + 1 < n && u.kind == 0 && e->uses[i + 1].kind == 2 && e->uses[i + 1].layer == l;
+    const bool bwd_after_fwd = i > 0 && u.kind == 2 && e->uses[i - 1].kind == 0 && e->uses[i - 1].layer == l;
     if (u.kind == 0) {
       // inside the last segment the forward keeps its activations in the segment buffers
       const int a_last = (e->S - 1) * e->K;
       const mt_bf16* xin = (l > a_last) ? e->seg[l - a_last - 1] : x_loc(e, l, x0, y_top);
       mt_bf16* xout = (l + 1 < e->L && l + 1 > a_last) ? e->seg[l - a_last] : x_loc(e, l + 1, x0, y_top);
-      status = mt_layer_fwd(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs);
+      status = layer_fwd_keep(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs,
+                              fwd_then_bwd);
       e->st.layer_fwd_calls++;
     } else if (u.kind == 1) {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
@@ -442,7 +449,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         if (status != MT_OK) break;
       }
       status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
-                                      e->lws_bytes, e->cs, e->mlp_done[jb]);
+                                      e->lws_bytes, e->cs, e->mlp_done[jb], bwd_after_fwd);
       e->st.layer_bwd_calls++;
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
       if (status == MT_OK) {

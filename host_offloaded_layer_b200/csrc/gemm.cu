@@ -455,6 +455,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // CTAs' empty / accumulator-full barriers, and both CTAs' epilogue warps
 // arrive on the even CTA's accumulator-empty barrier. No TMA load uses
 // cluster multicast: every CTA loads its own operands.
+// NH = 2 widens the pair tile to 256 x 512 (two N = 256 MMAs per K step into
+// one 512-column accumulator, four stages of 64-wide K, eight epilogue
+// warps): a quarter fewer operand bytes per FLOP and a deeper ring, at the
+// price of a single accumulator, whose epilogue the next tile's MMAs wait for.
 namespace c2 {
 constexpr int BM = 256, BN = 256;
 constexpr int HALF = 128 * 64 * 2;  // 16 KiB: one CTA's 128 rows of A (or B) for one 64-wide K atom
@@ -519,50 +523,51 @@ __host__ __device__ constexpr uint32_t make_idesc2(bool a_mn, bool b_mn) {
          (static_cast<uint32_t>(c2::BN >> 3) << 17) | (static_cast<uint32_t>(c2::BM >> 4) << 24);
 }
 
-// Bytes one CTA of the pair loads for one 64-wide K atom (boxes wholly past M
-// or N are skipped).
-__device__ __forceinline__ uint32_t half_bytes(bool a_mn, bool b_mn, int m0, int n0, int M, int N) {
+// Bytes one CTA loads for 128 rows of one operand and one 64-wide K atom
+// (boxes wholly past the operand's rows are skipped).
+__device__ __forceinline__ uint32_t rows_bytes(bool mn, int r0, int R) {
   uint32_t b = 0;
-  if (!a_mn) {
-    if (m0 < M) b += c2::HALF;
+  if (!mn) {
+    if (r0 < R) b += c2::HALF;
   } else {
     for (int j = 0; j < 2; ++j)
-      if (m0 + 64 * j < M) b += MN_BOX;
-  }
-  if (!b_mn) {
-    if (n0 < N) b += c2::HALF;
-  } else {
-    for (int j = 0; j < 2; ++j)
-      if (n0 + 64 * j < N) b += MN_BOX;
+      if (r0 + 64 * j < R) b += MN_BOX;
   }
   return b;
 }
 
-// KA: 64-wide K atoms per pipeline stage (1: 6 stages of 64, 2: 3 stages of 128).
-template <bool A_MN, bool B_MN, int KA>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+constexpr int threads2(int nh) { return 64 + 128 * nh; }
+
+// KA: 64-wide K atoms per pipeline stage (NH = 1: 1 -> 6 stages of 64, 2 -> 3
+// stages of 128; NH = 2: 1 -> 4 stages of 64). NH: N = 256 halves of the tile.
+template <bool A_MN, bool B_MN, int KA, int NH>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, EpiArgs ep,
                  int32_t* err) {
-  constexpr int BM = c2::BM, BN = c2::BN, BK = 64 * KA, STAGES = 6 / KA, HALF = c2::HALF;
-  constexpr int SMEM_TILES = c2::SMEM_TILES;
-  constexpr int STAGE_HALF = HALF * KA;  // one CTA's A (or B) bytes per stage
+  constexpr int BM = c2::BM, BN = 256 * NH, BK = 64 * KA, HALF = c2::HALF;
+  constexpr int STAGES = (NH == 1 ? 6 : 4) / KA;
+  constexpr int A_STAGE = HALF * KA, B_STAGE = HALF * KA * NH;  // one CTA's A / B bytes per stage
+  constexpr int NACC = NH == 1 ? 2 : 1;                           // accumulators in TMEM
+  constexpr int EPI_WARPS = 4 * NH;
+  constexpr int SMEM_TILES = STAGES * (A_STAGE + B_STAGE);
+  static_assert(SMEM_TILES == c2::SMEM_TILES, "every variant stages 192 KiB");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * STAGE_HALF;
+  uint8_t* sB = smem + STAGES * A_STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
   uint64_t* full = bars;                // TMA (both CTAs) -> MMA; used in the even CTA
   uint64_t* empty = bars + STAGES;      // MMA -> TMA, in each CTA
   uint64_t* tfull = bars + 2 * STAGES;  // MMA -> epilogue, in each CTA
-  uint64_t* tempty = tfull + 2;         // epilogues of both CTAs -> MMA; used in the even CTA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + NACC;      // epilogue warps of both CTAs -> MMA; used in the even CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + NACC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int num_m = (ep.M + BM - 1) / BM;
-  const int num_n = ep.swiglu == 1 ? (ep.F + 127) / 128 : (ep.N + BN - 1) / BN;
+  const int num_n = ep.swiglu == 1 ? (ep.F + 128 * NH - 1) / (128 * NH) : (ep.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (ep.K + BK - 1) / BK;
 
@@ -571,9 +576,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 2 * 128);
+      mbar_init(smem_u32(&tempty[b]), 2 * EPI_WARPS);  // one arrival per epilogue warp of each CTA
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -600,10 +605,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       int mb, nb;
       tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       const int m_own = mb * BM + static_cast<int>(rank) * 128;  // this CTA's A rows
-      // this CTA's B rows (SwiGLU: the gate rows in the even CTA, the up rows in the odd one)
-      const int n_base0 = ep.swiglu == 1 ? nb * 128 : nb * BN;
-      const int n_base1 = ep.swiglu == 1 ? ep.F + nb * 128 : nb * BN + 128;
-      const int n_own = rank == 0 ? n_base0 : n_base1;
+      // this CTA's B rows of N-half h (SwiGLU: the gate rows in the even CTA, the up rows in the odd one)
+      auto n_base = [&](int h, int rk) {
+        if (ep.swiglu == 1) return (rk == 0 ? 0 : ep.F) + nb * 128 * NH + h * 128;
+        return nb * BN + h * 256 + rk * 128;
+      };
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
@@ -616,12 +622,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const int k0 = kb * BK;
           const int atoms = min(KA, (ep.K - k0 + 63) / 64);  // atoms wholly past K are not loaded
           if (rank == 0) {
-            const uint32_t bytes = (half_bytes(A_MN, B_MN, mb * BM, n_base0, ep.M, ep.N) +
-                                    half_bytes(A_MN, B_MN, mb * BM + 128, n_base1, ep.M, ep.N)) *
-                                   static_cast<uint32_t>(atoms);
-            mbar_expect_tx(smem_u32(&full[s]), bytes);
+            uint32_t bytes = rows_bytes(A_MN, mb * BM, ep.M) + rows_bytes(A_MN, mb * BM + 128, ep.M);
+            for (int h = 0; h < NH; ++h) bytes += rows_bytes(B_MN, n_base(h, 0), ep.N) + rows_bytes(B_MN, n_base(h, 1), ep.N);
+            mbar_expect_tx(smem_u32(&full[s]), bytes * static_cast<uint32_t>(atoms));
           }
-          const uint32_t a_dst = smem_u32(sA + s * STAGE_HALF), b_dst = smem_u32(sB + s * STAGE_HALF);
+          const uint32_t a_dst = smem_u32(sA + s * A_STAGE), b_dst0 = smem_u32(sB + s * B_STAGE);
           for (int at = 0; at < atoms; ++at) {
             const int ka = k0 + 64 * at;
             if (!A_MN) {
@@ -631,12 +636,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (m_own + 64 * j < ep.M)
                   tma_load_2d_pair(a_dst + j * KA * MN_BOX + at * MN_BOX, &tmA, fb, m_own + 64 * j, ka);
             }
-            if (!B_MN) {
-              if (n_own < ep.N) tma_load_2d_pair(b_dst + at * HALF, &tmB, fb, ka, n_own);
-            } else {
-              for (int j = 0; j < 2; ++j)
-                if (n_own + 64 * j < ep.N)
-                  tma_load_2d_pair(b_dst + j * KA * MN_BOX + at * MN_BOX, &tmB, fb, n_own + 64 * j, ka);
+            for (int h = 0; h < NH; ++h) {
+              const int n_own = n_base(h, static_cast<int>(rank));
+              const uint32_t b_dst = b_dst0 + h * HALF * KA;  // sub-tile of N-half h
+              if (!B_MN) {
+                if (n_own < ep.N) tma_load_2d_pair(b_dst + at * HALF, &tmB, fb, ka, n_own);
+              } else {
+                for (int j = 0; j < 2; ++j)
+                  if (n_own + 64 * j < ep.N)
+                    tma_load_2d_pair(b_dst + j * KA * MN_BOX + at * MN_BOX, &tmB, fb, n_own + 64 * j, ka);
+              }
             }
           }
         }
@@ -651,8 +660,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       int tl = 0;
       bool ok = true;
       for (int t = cluster; t < num_tiles && ok; t += n_clusters, ++tl) {
-        const int ab = tl & 1;
-        const uint32_t aph = (tl >> 1) & 1u;
+        const int ab = NACC == 2 ? (tl & 1) : 0;
+        const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
         if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
         fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
@@ -665,7 +674,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           }
           fence_after();
           if (lane == 0) {
-            const uint32_t a_base = smem_u32(sA + s * STAGE_HALF), b_base = smem_u32(sB + s * STAGE_HALF);
+            const uint32_t a_base = smem_u32(sA + s * A_STAGE), b_base = smem_u32(sB + s * B_STAGE);
             const int ksteps = 4 * min(KA, (ep.K - kb * BK + 63) / 64);
             for (int kk = 0; kk < ksteps; ++kk) {
               // K-major: atom kk/4, then 16 elements (32 bytes) per step inside the swizzled row.
@@ -673,8 +682,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               const uint32_t koff_k = static_cast<uint32_t>((kk >> 2) * HALF + (kk & 3) * 32);
               const uint32_t koff_mn = static_cast<uint32_t>(kk * 2048);
               const uint64_t ad = A_MN ? smem_desc(a_base + koff_mn, KA * MN_BOX, 1024) : smem_desc(a_base + koff_k, 16, 1024);
-              const uint64_t bd = B_MN ? smem_desc(b_base + koff_mn, KA * MN_BOX, 1024) : smem_desc(b_base + koff_k, 16, 1024);
-              umma2_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+              for (int h = 0; h < NH; ++h) {
+                const uint32_t bh = b_base + h * HALF * KA;
+                const uint64_t bd = B_MN ? smem_desc(bh + koff_mn, KA * MN_BOX, 1024) : smem_desc(bh + koff_k, 16, 1024);
+                umma2_bf16(d_tmem + h * 256, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              }
             }
             umma2_commit_both(smem_u32(&empty[s]));
           }
@@ -687,20 +700,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
-    const int q = warp & 3;
+    const int q = warp & 3;          // TMEM lanes [32 q, 32 q + 32)
+    const int hc = (warp - 2) >> 2;  // N-half of the accumulator this warp drains
     int tl = 0;
     for (int t = cluster; t < num_tiles; t += n_clusters, ++tl) {
-      const int ab = tl & 1;
-      const uint32_t aph = (tl >> 1) & 1u;
+      const int ab = NACC == 2 ? (tl & 1) : 0;
+      const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
       int mb, nb;
       tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN + hc * 256);
       if (ep.swiglu == 1) {
         for (int c = 0; c < 4; ++c) {
-          const int f0 = nb * 128 + c * 32;
+          const int f0 = nb * 128 * NH + hc * 128 + c * 32;
           if (f0 >= ep.F) break;
           uint32_t rg[32], ru[32];
           tmem_ld32(tbase + static_cast<uint32_t>(c * 32), rg);
@@ -708,8 +723,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (row < ep.M) store_swiglu(ep, row, f0, rg, ru);
         }
       } else {
-        for (int c = 0; c < BN / 32; ++c) {
-          const int col0 = nb * BN + c * 32;
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = nb * BN + hc * 256 + c * 32;
           if (col0 >= ep.N) break;
           uint32_t r[32];
           tmem_ld32(tbase + static_cast<uint32_t>(c * 32), r);
@@ -722,7 +737,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
       }
       fence_before();
-      mbar_arrive_remote(map_to_rank(smem_u32(&tempty[ab]), 0));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&tempty[ab]), 0));
     }
   }
 
@@ -783,7 +799,7 @@ mt_status launch_1sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs
 }
 
 // Largest number of 2-CTA clusters of gemm2_kernel that fit on the device at once.
-template <bool A_MN, bool B_MN, int KA>
+template <bool A_MN, bool B_MN, int KA, int NH>
 int max_pair_clusters() {
   static std::mutex mu;
   static int cache[64] = {0};
@@ -793,10 +809,10 @@ int max_pair_clusters() {
   if (cache[dev] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(threads2(NH), 1, 1);
     cfg.dynamicSmemBytes = c2::SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<A_MN, B_MN, KA>, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<A_MN, B_MN, KA, NH>, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       n = num_sms() / 2;
     }
@@ -805,21 +821,21 @@ int max_pair_clusters() {
   return cache[dev];
 }
 
-template <bool A_MN, bool B_MN, int KA>
+template <bool A_MN, bool B_MN, int KA, int NH>
 mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm2_kernel<A_MN, B_MN, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(gemm2_kernel<A_MN, B_MN, KA, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     c2::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return fail(MT_ERR_CUDA, "gemm2 smem attribute: %s", cudaGetErrorString(attr_err));
-  const int num_n = ep.swiglu == 1 ? (ep.F + 127) / 128 : (ep.N + c2::BN - 1) / c2::BN;
+  const int num_n = ep.swiglu == 1 ? (ep.F + 128 * NH - 1) / (128 * NH) : (ep.N + 256 * NH - 1) / (256 * NH);
   const int num_tiles = ((ep.M + c2::BM - 1) / c2::BM) * num_n;
-  const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN, KA>());
+  const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN, KA, NH>());
   int32_t* err = device_error_word();
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
-  gemm2_kernel<A_MN, B_MN, KA><<<2 * clusters, NUM_THREADS, c2::SMEM_BYTES, st>>>(ta, tb, ep, err);
+  gemm2_kernel<A_MN, B_MN, KA, NH><<<2 * clusters, threads2(NH), c2::SMEM_BYTES, st>>>(ta, tb, ep, err);
   return launch_check("gemm2_kernel");
 }
 
@@ -835,9 +851,21 @@ int gemm_katoms() {
   return v;
 }
 
+// The 256 x 512 pair tile (NH = 2) when MT_GEMM_WIDE=1 is set.
+bool gemm_wide() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MT_GEMM_WIDE");
+    v = (e && std::string(e) == "1") ? 1 : 0;
+  }
+  return v == 1;
+}
+
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
-  return gemm_katoms() == 2 ? launch_2sm_ka<A_MN, B_MN, 2>(ta, tb, ep, st) : launch_2sm_ka<A_MN, B_MN, 1>(ta, tb, ep, st);
+  if (gemm_wide()) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
+  return gemm_katoms() == 2 ? launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st)
+                            : launch_2sm_ka<A_MN, B_MN, 1, 1>(ta, tb, ep, st);
 }
 
 // Which kernel runs: the 2-SM kernel unless MT_GEMM_KERNEL=1sm is set (kept for

@@ -20,7 +20,9 @@ namespace mt {
 
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done);
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd);
+mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
+                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep);
 mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, int64_t, int, float, cudaStream_t);
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
@@ -144,6 +146,23 @@ uint64_t mt_layer_workspace_bytes(const mt_layer_cfg* cfg, int32_t B, int32_t T,
 
 mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
                        int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream) {
+  return layer_fwd_keep(cfg, w_dev, x, y, B, T, mlp_chunk, ws, ws_bytes, stream, false);
+}
+
+mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
+                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
+                                 uint64_t ws_bytes, void* stream) {
+  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr, false);
+}
+
+}  // extern "C"
+
+// The layer forward. With `keep` the workspace is left holding everything the
+// layer's backward would recompute (h1, qkv after RoPE, o, lse, x2, h2, and
+// with a single MLP chunk also g, u and m), so that a backward called right
+// after it on the same workspace and weights can skip the recompute.
+mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
+                             int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
   if (!w_dev || !x || !y || !ws) return fail(MT_ERR_INVALID_ARG, "layer_fwd: NULL pointer");
@@ -161,27 +180,22 @@ mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_b
   const mt_param_offsets& O = G.off;
   for (int64_t r0 = 0; r0 < M; r0 += Mc) {
     const int64_t rows = std::min(Mc, M - r0);
-    MT_TRY(mlp_up(G, w_dev, w.h2 + r0 * G.H, rows, w, false, st));
+    MT_TRY(mlp_up(G, w_dev, w.h2 + r0 * G.H, rows, w, keep && Mc == M, st));
     MT_TRY(gemm_launch(w.m, G.F, false, w_dev + O.wd, G.F, false, y + r0 * G.H, G.H, false, false, rows, G.H, G.F,
                        nullptr, w.x2 + r0 * G.H, G.H, st));
   }
   return MT_OK;
 }
 
-mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
-                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream) {
-  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr);
-}
-
-}  // extern "C"
-
 // The layer backward; when mlp_done is given it is recorded on the stream as
-// soon as the MLP weights' gradients (Wg, Wu, Wd) are final.
+// soon as the MLP weights' gradients (Wg, Wu, Wd) are final. With reuse_fwd
+// the workspace still holds what layer_fwd_keep(keep = true) left in it for
+// these weights and this x, and the recompute is skipped (the values are the
+// ones it would produce: every kernel is deterministic).
 mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x,
                                      const mt_bf16* dy, mt_bf16* dx, float* dw_dev, int32_t B, int32_t T,
                                      int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream,
-                                     cudaEvent_t mlp_done) {
+                                     cudaEvent_t mlp_done, bool reuse_fwd) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
   if (!w_dev || !x || !dy || !dx || !dw_dev || !ws) return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: NULL pointer");
@@ -200,7 +214,7 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
   const int H = static_cast<int>(G.H);
 
   // ---- recompute (R)
-  MT_TRY(attention_half(G, w_dev, x, B, T, w, st));
+  if (!reuse_fwd) MT_TRY(attention_half(G, w_dev, x, B, T, w, st));
 
   // ---- MLP backward, chunk by chunk in token order
   for (int64_t r0 = 0; r0 < M; r0 += Mc) {
@@ -208,7 +222,7 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
     const bool acc = r0 > 0;
     const mt_bf16* h2c = w.h2 + r0 * G.H;
     const mt_bf16* dyc = dy + r0 * G.H;
-    MT_TRY(mlp_up(G, w_dev, h2c, rows, w, true, st));
+    if (!(reuse_fwd && Mc == M)) MT_TRY(mlp_up(G, w_dev, h2c, rows, w, true, st));
     // dWd (+)= dy^T m
     MT_TRY(gemm_launch(dyc, G.H, true, w.m, G.F, true, dw_dev + O.wd, G.F, true, acc, G.H, G.F, rows, nullptr, nullptr,
                        0, st));

@@ -316,17 +316,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           for (int e = 0; e < 32; ++e) sv[ch * 32 + e] = __uint_as_float(u[e]);
         }
         const int k0 = j * BKV + g * 64;
-        float mx = -INFINITY;
         if (k0 + 63 > q0) {  // a block on the diagonal: keys after the row are masked
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
+          for (int e = 0; e < 64; ++e)
             if (k0 + e > q_row) sv[e] = -INFINITY;
-            mx = fmaxf(mx, sv[e]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, sv[e]);
         }
+        // row maximum over eight independent partial maxima (short dependency chains)
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = sv[e];
+#pragma unroll
+        for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], sv[e]);
+        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         mx *= scale_log2;
         // rescale O_g only when some row of the warp raised its maximum by more than the threshold
         if (__any_sync(0xffffffffu, mx > m_run + RESCALE_THRESHOLD)) {
@@ -356,15 +357,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         // P over the S values just read (its MMA reader of two blocks ago finished before S_i was
         // written: the tensor core runs the CTA's MMAs in order and s_full covers all earlier ones)
         const float mb = m_run == -INFINITY ? 0.f : m_run;  // a fully masked row half gives P = 0
-        float lsum = 0.f;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight partial sums, added in a fixed tree
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float p0 = ex2(fmaf(sv[2 * e], scale_log2, -mb));
           const float p1 = ex2(fmaf(sv[2 * e + 1], scale_log2, -mb));
-          lsum += p0 + p1;
+          l8[e & 7] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }
+        const float lsum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         tmem_st32(tmem + lane_base + COL_S0 + s * BKV + g * 64, pk);
         l_run += lsum;
         fence_before();
@@ -694,16 +696,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
       }
-      const float* L2 = lsd + sq * 128 + g * 32;
-      const float* Dl = L2 + 64;
+      // this group's 32 log-sum-exp and delta values (16-byte aligned: vector broadcast loads)
+      const float4* L4 = reinterpret_cast<const float4*>(lsd + sq * 128 + g * 32);
+      const float4* D4 = reinterpret_cast<const float4*>(lsd + sq * 128 + 64 + g * 32);
       const int qc0 = q0 + g * 32;
       const bool diag = qc0 < k0 + 127;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float p = ex2(fmaf(sv[e], scale_log2, -L2[e]));
-        if (diag && kv_row > qc0 + e) p = 0.f;
-        sv[e] = p;
-        dv[e] = p * (dv[e] - Dl[e]);
+      for (int v4 = 0; v4 < 8; ++v4) {
+        const float4 l4 = L4[v4], d4 = D4[v4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int e = v4 * 4 + c;
+          float p = ex2(fmaf(sv[e], scale_log2, -lv[c]));
+          if (diag && kv_row > qc0 + e) p = 0.f;
+          sv[e] = p;
+          dv[e] = p * (dv[e] - dl[c]);
+        }
       }
       {  // P^T and dS^T over the S^T / dP^T values just read
         uint32_t pp[16], pd[16];

@@ -851,19 +851,26 @@ int gemm_katoms() {
   return v;
 }
 
-// The 256 x 512 pair tile (NH = 2) when MT_GEMM_WIDE=1 is set.
-bool gemm_wide() {
-  static int v = -1;
-  if (v < 0) {
+// Pair-tile width. The 256 x 512 tile (NH = 2) measured 4-7% faster on the
+// weight-gradient layout (both operands MN-major, K = tokens >= 16384, fp32 out),
+// where a tile's main loop is long enough to hide its unbuffered epilogue, and
+// 2-5% slower on the forward and input-gradient shapes of the layer (K = 3584):
+// it is used for the weight-gradient layout with K >= 8192. MT_GEMM_WIDE=1 / 0
+// forces it on / off (comparison measurements).
+int gemm_wide_mode() {
+  static int v = -2;
+  if (v == -2) {
     const char* e = getenv("MT_GEMM_WIDE");
-    v = (e && std::string(e) == "1") ? 1 : 0;
+    v = !e ? -1 : (std::string(e) == "1" ? 1 : 0);
   }
-  return v == 1;
+  return v;
 }
 
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
-  if (gemm_wide()) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
+  const int mode = gemm_wide_mode();
+  const bool wide = mode == 1 || (mode == -1 && A_MN && B_MN && ep.swiglu == 0 && ep.K >= 8192);
+  if (wide) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
   return gemm_katoms() == 2 ? launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st)
                             : launch_2sm_ka<A_MN, B_MN, 1, 1>(ta, tb, ep, st);
 }

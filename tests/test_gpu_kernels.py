@@ -25,7 +25,8 @@ def _check_dev_error():
 
 # ------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
-@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 300, 136), (2048, 4096, 512), (96, 40, 1000)])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 300, 136), (2048, 4096, 512), (96, 40, 1000),
+                                   (600, 1100, 8200)])  # K >= 8192: the 256 x 512 tile on the MN / MN layout
 def test_gemm_layouts_match_fp64_matmul(a_mn, b_mn, M, N, K):
     import torch
     lda = ((M if a_mn else K) + 7) // 8 * 8 + 8

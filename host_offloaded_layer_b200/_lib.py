@@ -161,6 +161,11 @@ def last_error() -> str:
     return load().mt_last_error().decode(errors="replace")
 
 
+def mt_last_error() -> str:
+    """The calling thread's last error message (same as last_error())."""
+    return last_error()
+
+
 def _check(code: int) -> None:
     if code != 0:
         raise MTError(code, last_error())
@@ -342,6 +347,10 @@ def mt_engine_destroy(engine):
     load().mt_engine_destroy(engine)
 
 
+def mt_schedule_len(n_layers, K) -> int:
+    return load().mt_schedule_len(n_layers, K)
+
+
 def mt_schedule(n_layers, K, n_slots):
     n = load().mt_schedule_len(n_layers, K)
     arrs = [(c_i32 * n)() for _ in range(4)]
@@ -361,6 +370,11 @@ def mt_host_optimizer_create(store, cfg) -> int:
 
 def mt_host_optimizer_destroy(opt):
     load().mt_host_optimizer_destroy(opt)
+
+
+def mt_host_optimizer_sink(layer, grad, n, opt):
+    """Applies one layer's gradient record (host fp32, n elements) to the optimizer `opt` directly."""
+    _check(load().mt_host_optimizer_sink(layer, ctypes.cast(_ptr(grad), ctypes.POINTER(c_f32)), n, opt))
 
 
 def optimizer_sink():

@@ -108,6 +108,15 @@ def test_schedule_holds_each_layer_when_used(n_layers, K, R):
         assert loads == n_layers
 
 
+def test_python_binding_has_every_declared_entry_point():
+    """The binding offers a function of the same name for every call the header declares."""
+    decl = set(re.findall(r"\b(?:mt_status|uint64_t|int32_t|void|float|mt_bf16|char)\s*\*?\s*(mt_[a-z0-9_]+)\s*\(",
+                          open(os.path.join(ROOT, "include", "mt.h")).read()))
+    missing = sorted(n for n in decl if not callable(getattr(L, n, None)))
+    assert not missing, missing
+    assert L.mt_schedule_len(4, 4) == len(L.mt_schedule(4, 4, 4)[0])
+
+
 def test_invalid_arguments_are_rejected_without_a_gpu():
     with pytest.raises(L.MTError) as e:
         L.mt_layer_param_offsets(L.make_cfg(256, 4, 3, 64, 688))

@@ -50,6 +50,10 @@ CONFIGS = {
     3: dict(name="qwen2.5-7b-shape_x28_b96x1024", shape=QWEN7B, L=28, B=96, T=1024, K=4, chunk=0),
     4: dict(name="qwen2.5-14b-shape_x48_b64x1024", shape=QWEN14B, L=48, B=64, T=1024, K=4, chunk=0),
     5: dict(name="qwen2.5-7b-shape_x28_b1x32768_mlpchunk4096", shape=QWEN7B, L=28, B=1, T=32768, K=4, chunk=4096),
+    # MegaTrain Table 7's 128K-context row (B = 1, chunked MLP): the long-context regime, beyond the hot-path
+    # workloads above; one step takes tens of seconds
+    6: dict(name="qwen2.5-7b-shape_x28_b1x131072_mlpchunk4096", shape=QWEN7B, L=28, B=1, T=131072, K=4,
+            chunk=4096),
 }
 # The ablations of MegaTrain Table 4, as engine options.
 ABLATIONS = {

@@ -40,10 +40,12 @@ struct Use {
 std::vector<Use> build_uses(int L, int K);
 void plan_slots(const std::vector<Use>& u, int R, std::vector<int>& slot, std::vector<int>& load);
 mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
-                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep);
+                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep,
+                         cudaEvent_t mlp_weights);
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd);
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd,
+                                 cudaEvent_t wd_done);
 }  // namespace mt
 
 using namespace mt;
@@ -206,6 +208,8 @@ struct mt_engine {
   std::vector<Use> uses;
   std::vector<int> uslot, uload, prev_of_slot, load_of_use;
   std::vector<cudaEvent_t> ready, done, g_ready, d2h_done, mlp_done;
+  std::vector<cudaEvent_t> ready_attn;  // per use: the record's head (g1 .. g2) is on the device
+  std::vector<cudaEvent_t> wd_done;     // per backward: the down projection's gradient is final
   cudaEvent_t fin = nullptr;
   bool resident_loaded = false;
   int64_t h2d_count = 0;
@@ -388,8 +392,14 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       }
       if (p >= 0) MT_CUDA(cudaStreamWaitEvent(e->ps, e->done[p], 0));
       const int layer = e->uses[next_load].layer;
-      MT_CUDA(cudaMemcpyAsync(e->slot[e->uslot[next_load]], mt_host_store_bf16(store, layer), rec * 2,
-                              cudaMemcpyHostToDevice, e->ps));
+      // two pieces: the record's head (g1 .. g2, all the attention half reads) first, so that a
+      // forward can start its attention while the MLP weights are still crossing the link
+      const uint64_t head = e->G.off.wg;
+      mt_bf16* dst = e->slot[e->uslot[next_load]];
+      const mt_bf16* src = mt_host_store_bf16(store, layer);
+      MT_CUDA(cudaMemcpyAsync(dst, src, head * 2, cudaMemcpyHostToDevice, e->ps));
+      MT_CUDA(cudaEventRecord(e->ready_attn[next_load], e->ps));
+      MT_CUDA(cudaMemcpyAsync(dst + head, src + head, (rec - head) * 2, cudaMemcpyHostToDevice, e->ps));
       MT_CUDA(cudaEventRecord(e->ready[next_load], e->ps));
       ++e->h2d_count;
       e->st.h2d_bytes += rec * 2;
@@ -418,8 +428,17 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
     const int l = u.layer;
     const int s = l / e->K, a = s * e->K;
     mt_bf16* w = e->slot[e->uslot[i]];
+    // a forward waits for the record's head and hands the full-record event to the layer, which
+    // waits for it before its MLP; a backward waits for the whole record
+    cudaEvent_t mlp_weights = nullptr;
     if (!skip_loads && e->load_of_use[i] >= 0) {
-      status = cuda_check(cudaStreamWaitEvent(e->cs, e->ready[e->load_of_use[i]], 0), "wait weights");
+      const int ld = e->load_of_use[i];
+      if (u.kind == 2) {
+        status = cuda_check(cudaStreamWaitEvent(e->cs, e->ready[ld], 0), "wait weights");
+      } else {
+        status = cuda_check(cudaStreamWaitEvent(e->cs, e->ready_attn[ld], 0), "wait weights");
+        mlp_weights = e->ready[ld];
+      }
       if (status != MT_OK) break;
     }
     // the backward of a layer that directly follows its own forward (the top layer) finds
@@ -432,12 +451,12 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       const mt_bf16* xin = (l > a_last) ? e->seg[l - a_last - 1] : x_loc(e, l, x0, y_top);
       mt_bf16* xout = (l + 1 < e->L && l + 1 > a_last) ? e->seg[l - a_last] : x_loc(e, l + 1, x0, y_top);
       status = layer_fwd_keep(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs,
-                              fwd_then_bwd);
+                              fwd_then_bwd, mlp_weights);
       e->st.layer_fwd_calls++;
     } else if (u.kind == 1) {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
-      status = mt_layer_fwd(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes,
-                            e->cs);
+      status = layer_fwd_keep(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes,
+                              e->cs, false, mlp_weights);
       e->st.layer_fwd_calls++;
     } else {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
@@ -449,7 +468,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         if (status != MT_OK) break;
       }
       status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
-                                      e->lws_bytes, e->cs, e->mlp_done[jb], bwd_after_fwd);
+                                      e->lws_bytes, e->cs, e->mlp_done[jb], bwd_after_fwd, e->wd_done[jb]);
       e->st.layer_bwd_calls++;
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
       if (status == MT_OK) {
@@ -475,12 +494,17 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
             dst = e->slab[p];
           }
         }
-        // two pieces: the MLP weights' gradients (the record's tail from Wg on) as soon as
-        // the MLP backward is done, then the rest when the layer is done
-        const uint64_t split = e->G.off.wg;
+        // three pieces, each as soon as it is final: the down projection's gradient (the record's
+        // tail from Wd on), then the gate / up projections' (Wg, Wu), then the rest when the layer is done
+        const uint64_t split = e->G.off.wg, split_d = e->G.off.wd;
+        if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->wd_done[jb], 0), "wait wd_done");
+        if (status == MT_OK)
+          status = cuda_check(cudaMemcpyAsync(dst + split_d, e->dgrad[ns] + split_d, (rec - split_d) * 4,
+                                              cudaMemcpyDeviceToHost, e->os),
+                              "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->mlp_done[jb], 0), "wait mlp_done");
         if (status == MT_OK)
-          status = cuda_check(cudaMemcpyAsync(dst + split, e->dgrad[ns] + split, (rec - split) * 4,
+          status = cuda_check(cudaMemcpyAsync(dst + split, e->dgrad[ns] + split, (split_d - split) * 4,
                                               cudaMemcpyDeviceToHost, e->os),
                               "gradient D2H");
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->g_ready[jb], 0), "wait g_ready");
@@ -602,6 +626,8 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
     return MT_OK;
   };
   mt_status s = mk(e->ready, n);
+  if (s == MT_OK) s = mk(e->ready_attn, n);
+  if (s == MT_OK) s = mk(e->wd_done, n_layers);
   if (s == MT_OK) s = mk(e->done, n);
   if (s == MT_OK) s = mk(e->g_ready, n_layers);
   if (s == MT_OK) s = mk(e->d2h_done, n_layers);
@@ -729,7 +755,8 @@ void mt_engine_destroy(mt_engine* e) {
   cudaStreamSynchronize(e->cs);
   cudaStreamSynchronize(e->ps);
   cudaStreamSynchronize(e->os);
-  for (auto* v : {&e->ready, &e->done, &e->g_ready, &e->d2h_done, &e->mlp_done, &e->timer.ev})
+  for (auto* v : {&e->ready, &e->ready_attn, &e->wd_done, &e->done, &e->g_ready, &e->d2h_done, &e->mlp_done,
+                  &e->timer.ev})
     for (auto ev : *v)
       if (ev) cudaEventDestroy(ev);
   if (e->fin) cudaEventDestroy(e->fin);

@@ -20,9 +20,11 @@ namespace mt {
 
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd);
+                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd,
+                                 cudaEvent_t wd_done);
 mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
-                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep);
+                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep,
+                         cudaEvent_t mlp_weights);
 mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, int64_t, int, float, cudaStream_t);
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
@@ -146,13 +148,14 @@ uint64_t mt_layer_workspace_bytes(const mt_layer_cfg* cfg, int32_t B, int32_t T,
 
 mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
                        int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream) {
-  return layer_fwd_keep(cfg, w_dev, x, y, B, T, mlp_chunk, ws, ws_bytes, stream, false);
+  return layer_fwd_keep(cfg, w_dev, x, y, B, T, mlp_chunk, ws, ws_bytes, stream, false, nullptr);
 }
 
 mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
                                  uint64_t ws_bytes, void* stream) {
-  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr, false);
+  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr, false,
+                                nullptr);
 }
 
 }  // extern "C"
@@ -160,9 +163,12 @@ mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, 
 // The layer forward. With `keep` the workspace is left holding everything the
 // layer's backward would recompute (h1, qkv after RoPE, o, lse, x2, h2, and
 // with a single MLP chunk also g, u and m), so that a backward called right
-// after it on the same workspace and weights can skip the recompute.
+// after it on the same workspace and weights can skip the recompute. When
+// `mlp_weights` is given the stream waits for it between the attention half
+// and the MLP (the streaming engine uploads a record in two pieces).
 mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
-                             int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep) {
+                             int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep,
+                             cudaEvent_t mlp_weights) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
   if (!w_dev || !x || !y || !ws) return fail(MT_ERR_INVALID_ARG, "layer_fwd: NULL pointer");
@@ -177,6 +183,7 @@ mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, cons
                             (unsigned long long)bp.used);
   cudaStream_t st = as_stream(stream);
   MT_TRY(attention_half(G, w_dev, x, B, T, w, st));
+  if (mlp_weights) MT_CUDA(cudaStreamWaitEvent(st, mlp_weights, 0));
   const mt_param_offsets& O = G.off;
   for (int64_t r0 = 0; r0 < M; r0 += Mc) {
     const int64_t rows = std::min(Mc, M - r0);
@@ -195,7 +202,7 @@ mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, cons
 mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x,
                                      const mt_bf16* dy, mt_bf16* dx, float* dw_dev, int32_t B, int32_t T,
                                      int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream,
-                                     cudaEvent_t mlp_done, bool reuse_fwd) {
+                                     cudaEvent_t mlp_done, bool reuse_fwd, cudaEvent_t wd_done) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
   if (!w_dev || !x || !dy || !dx || !dw_dev || !ws) return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: NULL pointer");
@@ -226,6 +233,7 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
     // dWd (+)= dy^T m
     MT_TRY(gemm_launch(dyc, G.H, true, w.m, G.F, true, dw_dev + O.wd, G.F, true, acc, G.H, G.F, rows, nullptr, nullptr,
                        0, st));
+    if (wd_done && r0 + rows >= M) MT_CUDA(cudaEventRecord(wd_done, st));  // dWd is final after the last chunk
     if (swiglu_bwd_fused()) {
       // dm = dy Wd, and in the same GEMM's epilogue [dg|du] in place over [g|u]
       MT_TRY(gemm_swiglu_bwd_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.gu, 2 * G.F, rows, G.F, G.H, st));

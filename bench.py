@@ -76,23 +76,32 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def gemm_source_hash() -> str:
+    """SHA-256 of the GEMM's code (gemm.cu + tcgen05.cuh) with // comments, trailing
+    blanks and empty lines removed, so that an edit of comments alone keeps it."""
+    import hashlib
+    import re
+    csrc = os.path.join(ROOT, "host_offloaded_layer_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "tcgen05.cuh"):
+        lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in open(os.path.join(csrc, f)).read().splitlines())
+        h.update(("\n".join(ln for ln in lines if ln) + "\n").encode())
+    return h.hexdigest()
+
+
 def gemm_traffic(workload: str):
     """DRAM bytes per GEMM launch from the committed ncu summary, when that summary
-    was taken on this workload with the current GEMM source (else None)."""
-    import hashlib
+    was taken on this workload with the current GEMM code (else None)."""
     path = os.path.join(ROOT, "profiles", "gemm2_kernel_traffic.txt")
     if not os.path.exists(path):
         return None
     kv = {}
     for line in open(path):
-        if ":" in line:
+        if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    csrc = os.path.join(ROOT, "host_offloaded_layer_b200", "csrc")
-    h = hashlib.sha256()
-    for f in ("gemm.cu", "tcgen05.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    if kv.get("kernel_source_sha256") != h.hexdigest() or kv.get("workload") != workload:
+    h = gemm_source_hash()
+    if kv.get("kernel_code_sha256") != h or kv.get("workload") != workload:
         return None
     return float(kv["dram_bytes_per_launch"])
 

@@ -451,10 +451,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // rows of A and its own 128 columns' worth of B (6 stages of 32 KiB), so per
 // FLOP each SM moves a third less operand data through shared memory than the
 // one-SM 128 x 256 tile. The even CTA issues the MMAs for the pair; its full
-// barriers count both CTAs' TMA bytes, the MMA commits are multicast to both
-// CTAs' empty / accumulator-full barriers, and both CTAs' epilogue warps
-// arrive on the even CTA's accumulator-empty barrier. No TMA load uses
-// cluster multicast: every CTA loads its own operands.
+// barriers count both CTAs' TMA bytes, each MMA commit signals both CTAs'
+// empty / accumulator-full barriers, and both CTAs' epilogue warps arrive on
+// the even CTA's accumulator-empty barrier. Every CTA loads its own operands
+// with plain per-CTA tensor copies; no copy is shared between CTAs.
 // NH = 2 widens the pair tile to 256 x 512 (two N = 256 MMAs per K step into
 // one 512-column accumulator, four stages of 64-wide K, eight epilogue
 // warps): a quarter fewer operand bytes per FLOP and a deeper ring, at the

@@ -462,6 +462,19 @@ def run_ours(args, cfg, rank, world, local_rank):
                              "sample": cpu_desc},
             "device_workspace_gb": nbytes / 1e9,
         }
+    if args.trace:
+        # one more engine over the same memory, with the event timeline on: two steps, the last one's
+        # uploads, layer calls and offloads written to the trace file (outside every timed region)
+        L_.mt_engine_destroy(eng)
+        topts = L_.mt_engine_opts.from_buffer_copy(opts)
+        topts.trace = 1
+        eng = L_.mt_engine_create(lcfg, nL, B, T, topts, ws, nbytes, *streams)
+        for _ in range(2):
+            dev_step()
+        torch.cuda.synchronize()
+        if rank == 0:
+            with open(args.trace, "w") as f:
+                json.dump({"workload": cfg["name"], "intervals": L_.mt_engine_trace(eng)}, f, indent=0)
     L_.mt_engine_destroy(eng)
     if opt is not None:
         L_.mt_host_optimizer_destroy(opt)
@@ -482,6 +495,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--full-model", action="store_true",
                     help="add the embedding and the final norm + LM head + loss (vocabulary 152064) to the step")
+    ap.add_argument("--trace", default="", metavar="PATH",
+                    help="after the measurement, write the event timeline of one more step to PATH (JSON)")
     ap.add_argument("--sink", default="none", choices=["none", "adamw"],
                     help="what receives each layer's gradient record (adamw: the CPU optimizer step)")
     ap.add_argument("--ablation", default="none", choices=sorted(ABLATIONS),

@@ -44,7 +44,14 @@ class mt_param_offsets(ctypes.Structure):
 class mt_engine_opts(ctypes.Structure):
     _fields_ = [(n, c_i32) for n in ("ckpt_interval", "n_weight_slots", "n_host_slabs", "n_dev_grad_slabs",
                                      "mlp_chunk", "resident", "timeout_ms", "fail_h2d_at", "time_gemms",
-                                     "no_slab_pool")]
+                                     "no_slab_pool", "trace")]
+
+
+class mt_trace_rec(ctypes.Structure):
+    _fields_ = [("kind", c_i32), ("layer", c_i32), ("begin_ms", c_f32), ("end_ms", c_f32)]
+
+
+TRACE_KINDS = ("h2d", "forward", "reforward", "backward", "d2h")
 
 
 class mt_stats(ctypes.Structure):
@@ -102,6 +109,7 @@ _SIGS = {
     "mt_stream_step": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp]),
     "mt_stream_step_hooked": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp, mt_head_hook, c_vp]),
     "mt_stream_step_host": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp]),
+    "mt_engine_trace": (c_i32, [c_vp, ctypes.POINTER(mt_trace_rec), c_i32, ctypes.POINTER(c_i32)]),
     "mt_engine_stats": (c_i32, [c_vp, ctypes.POINTER(mt_stats)]),
     "mt_engine_reset": (c_i32, [c_vp]),
     "mt_engine_destroy": (None, [c_vp]),
@@ -295,9 +303,9 @@ def mt_host_store_destroy(store):
 
 
 def make_opts(ckpt_interval=4, n_weight_slots=0, n_host_slabs=0, n_dev_grad_slabs=0, mlp_chunk=0, resident=0,
-              timeout_ms=0, fail_h2d_at=0, time_gemms=0, no_slab_pool=0) -> mt_engine_opts:
+              timeout_ms=0, fail_h2d_at=0, time_gemms=0, no_slab_pool=0, trace=0) -> mt_engine_opts:
     return mt_engine_opts(ckpt_interval, n_weight_slots, n_host_slabs, n_dev_grad_slabs, mlp_chunk, resident,
-                          timeout_ms, fail_h2d_at, time_gemms, no_slab_pool)
+                          timeout_ms, fail_h2d_at, time_gemms, no_slab_pool, trace)
 
 
 def mt_engine_workspace_bytes(cfg, n_layers, B, T, opts) -> int:
@@ -337,6 +345,15 @@ def mt_engine_stats(engine) -> mt_stats:
     s = mt_stats()
     _check(load().mt_engine_stats(engine, ctypes.byref(s)))
     return s
+
+
+def mt_engine_trace(engine, cap=4096) -> list:
+    """The last step's timeline: [{kind, layer, begin_ms, end_ms}] in issue order."""
+    recs = (mt_trace_rec * cap)()
+    n = c_i32(0)
+    _check(load().mt_engine_trace(engine, recs, cap, ctypes.byref(n)))
+    return [{"kind": TRACE_KINDS[r.kind], "layer": r.layer, "begin_ms": r.begin_ms, "end_ms": r.end_ms}
+            for r in recs[:min(n.value, cap)]]
 
 
 def mt_engine_reset(engine):

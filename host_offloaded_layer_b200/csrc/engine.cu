@@ -211,6 +211,15 @@ struct mt_engine {
   std::vector<cudaEvent_t> ready_attn;  // per use: the record's head (g1 .. g2) is on the device
   std::vector<cudaEvent_t> wd_done;     // per backward: the down projection's gradient is final
   cudaEvent_t fin = nullptr;
+  // timeline (opts.trace): timing events, the step's start, and (kind, layer, begin, end) slots
+  struct TraceSlot {
+    int kind, layer, eb, ee;
+  };
+  std::vector<cudaEvent_t> tr_ev;
+  cudaEvent_t tr_t0 = nullptr;
+  std::vector<TraceSlot> tr;
+  int tr_used = 0;
+  bool tr_valid = false;
   bool resident_loaded = false;
   int64_t h2d_count = 0;
   EventTimer timer;
@@ -231,6 +240,7 @@ mt_status validate_opts(const mt_engine_opts* in, int L, mt_engine_opts* o) {
   *o = *in;
   if (o->ckpt_interval < 1) return fail(MT_ERR_INVALID_ARG, "ckpt_interval must be >= 1");
   if (o->no_slab_pool < 0) return fail(MT_ERR_INVALID_ARG, "no_slab_pool must be 0 or 1");
+  if (o->trace < 0 || o->trace > 1) return fail(MT_ERR_INVALID_ARG, "trace must be 0 or 1");
   if (o->n_weight_slots < 0 || o->n_host_slabs < 0 || o->n_dev_grad_slabs < 0 || o->mlp_chunk < 0 ||
       o->timeout_ms < 0 || o->fail_h2d_at < 0)
     return fail(MT_ERR_INVALID_ARG, "engine options must be >= 0");
@@ -363,6 +373,34 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
   mt_status status = MT_OK;
   const auto timeout = std::chrono::milliseconds(e->opts.timeout_ms);
 
+  // timeline: begin / end events of one interval on a stream (no-ops without opts.trace, and
+  // once the event pool is used up)
+  const bool tracing = e->opts.trace != 0;
+  e->tr.clear();
+  e->tr_used = 0;
+  e->tr_valid = false;
+  auto tr_begin = [e, tracing](int kind, int layer, cudaStream_t stream) -> int {
+    if (!tracing || e->tr_used + 2 > static_cast<int>(e->tr_ev.size())) return -1;
+    const int k = static_cast<int>(e->tr.size());
+    e->tr.push_back({kind, layer, e->tr_used, e->tr_used + 1});
+    e->tr_used += 2;
+    if (cudaEventRecord(e->tr_ev[e->tr[k].eb], stream) != cudaSuccess) {
+      cudaGetLastError();
+      e->tr.pop_back();
+      return -1;
+    }
+    return k;
+  };
+  auto tr_end = [e](int k, cudaStream_t stream) {
+    if (k < 0) return;
+    if (cudaEventRecord(e->tr_ev[e->tr[k].ee], stream) != cudaSuccess) cudaGetLastError();
+  };
+  if (tracing) {  // the step's time origin, ahead of everything on all three streams
+    MT_CUDA(cudaEventRecord(e->tr_t0, e->cs));
+    MT_CUDA(cudaStreamWaitEvent(e->ps, e->tr_t0, 0));
+    MT_CUDA(cudaStreamWaitEvent(e->os, e->tr_t0, 0));
+  }
+
   // sink thread for this step
   {
     std::lock_guard<std::mutex> lk(e->mu);
@@ -397,10 +435,12 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       const uint64_t head = e->G.off.wg;
       mt_bf16* dst = e->slot[e->uslot[next_load]];
       const mt_bf16* src = mt_host_store_bf16(store, layer);
+      const int tk = tr_begin(0, layer, e->ps);
       MT_CUDA(cudaMemcpyAsync(dst, src, head * 2, cudaMemcpyHostToDevice, e->ps));
       MT_CUDA(cudaEventRecord(e->ready_attn[next_load], e->ps));
       MT_CUDA(cudaMemcpyAsync(dst + head, src + head, (rec - head) * 2, cudaMemcpyHostToDevice, e->ps));
       MT_CUDA(cudaEventRecord(e->ready[next_load], e->ps));
+      tr_end(tk, e->ps);
       ++e->h2d_count;
       e->st.h2d_bytes += rec * 2;
       e->st.weight_loads += 1;
@@ -445,6 +485,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
     // the forward's internals still in the layer workspace and skips their recompute
     const bool fwd_then_bwd = i + 1 < n && u.kind == 0 && e->uses[i + 1].kind == 2 && e->uses[i + 1].layer == l;
     const bool bwd_after_fwd = i > 0 && u.kind == 2 && e->uses[i - 1].kind == 0 && e->uses[i - 1].layer == l;
+    const int tk = tr_begin(u.kind + 1, l, e->cs);
     if (u.kind == 0) {
       // inside the last segment the forward keeps its activations in the segment buffers
       const int a_last = (e->S - 1) * e->K;
@@ -453,11 +494,13 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       status = layer_fwd_keep(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs,
                               fwd_then_bwd, mlp_weights);
       e->st.layer_fwd_calls++;
+      tr_end(tk, e->cs);
     } else if (u.kind == 1) {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
       status = layer_fwd_keep(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes,
                               e->cs, false, mlp_weights);
       e->st.layer_fwd_calls++;
+      tr_end(tk, e->cs);
     } else {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
       const mt_bf16* dy = (jb == 0) ? dy_top : e->gbuf[(jb - 1) % 2];
@@ -470,6 +513,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
                                       e->lws_bytes, e->cs, e->mlp_done[jb], bwd_after_fwd, e->wd_done[jb]);
       e->st.layer_bwd_calls++;
+      tr_end(tk, e->cs);
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
       if (status == MT_OK) {
         // take a pinned slab from the pool (bounded wait), then offload. Without the pool
@@ -498,6 +542,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         // tail from Wd on), then the gate / up projections' (Wg, Wu), then the rest when the layer is done
         const uint64_t split = e->G.off.wg, split_d = e->G.off.wd;
         if (status == MT_OK) status = cuda_check(cudaStreamWaitEvent(e->os, e->wd_done[jb], 0), "wait wd_done");
+        const int tko = status == MT_OK ? tr_begin(4, l, e->os) : -1;
         if (status == MT_OK)
           status = cuda_check(cudaMemcpyAsync(dst + split_d, e->dgrad[ns] + split_d, (rec - split_d) * 4,
                                               cudaMemcpyDeviceToHost, e->os),
@@ -511,6 +556,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         if (status == MT_OK)
           status = cuda_check(
               cudaMemcpyAsync(dst, e->dgrad[ns], split * 4, cudaMemcpyDeviceToHost, e->os), "gradient D2H");
+        tr_end(tko, e->os);
         if (status == MT_OK) status = cuda_check(cudaEventRecord(e->d2h_done[jb], e->os), "record d2h_done");
         if (status == MT_OK) {
           e->st.d2h_bytes += rec * 4;
@@ -548,6 +594,7 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
     if (status == MT_OK) status = poll_event(e->fin, Clock::now() + timeout, "compute stream");
   }
   if (status == MT_OK && e->opts.resident) e->resident_loaded = true;
+  if (status == MT_OK && tracing) e->tr_valid = true;
   return status;
 }
 
@@ -633,6 +680,15 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
   if (s == MT_OK) s = mk(e->d2h_done, n_layers);
   if (s == MT_OK) s = mk(e->mlp_done, n_layers);
   if (s == MT_OK) s = cuda_check(cudaEventCreateWithFlags(&e->fin, cudaEventDisableTiming), "event");
+  if (s == MT_OK && o.trace) {
+    // two timing events per upload (at most one per use), layer call and offload
+    e->tr_ev.assign(2 * (2 * n + n_layers), nullptr);
+    for (auto& ev : e->tr_ev) {
+      s = cuda_check(cudaEventCreate(&ev), "trace event");
+      if (s != MT_OK) break;
+    }
+    if (s == MT_OK) s = cuda_check(cudaEventCreate(&e->tr_t0), "trace event");
+  }
   if (s == MT_OK && o.time_gemms) {
     e->timer.ev.assign(8192, nullptr);
     for (auto& ev : e->timer.ev) {
@@ -719,6 +775,22 @@ mt_status mt_engine_stats(const mt_engine* e, mt_stats* out) {
   return MT_OK;
 }
 
+mt_status mt_engine_trace(mt_engine* e, mt_trace_rec* out, int32_t cap, int32_t* n) {
+  if (!e || !n || cap < 0 || (cap > 0 && !out)) return fail(MT_ERR_INVALID_ARG, "engine_trace: bad argument");
+  if (!e->opts.trace || !e->tr_valid)
+    return fail(MT_ERR_INVALID_ARG, "engine_trace: the engine has no traced step (create it with trace = 1)");
+  const int avail = static_cast<int>(e->tr.size());
+  for (int k = 0; k < avail && k < cap; ++k) {
+    const auto& t = e->tr[k];
+    float b = 0.f, en = 0.f;
+    MT_CUDA(cudaEventElapsedTime(&b, e->tr_t0, e->tr_ev[t.eb]));
+    MT_CUDA(cudaEventElapsedTime(&en, e->tr_t0, e->tr_ev[t.ee]));
+    out[k] = {t.kind, t.layer, b, en};
+  }
+  *n = avail;
+  return MT_OK;
+}
+
 mt_status mt_engine_reset(mt_engine* e) {
   if (!e) return fail(MT_ERR_INVALID_ARG, "engine is NULL");
   const auto deadline = Clock::now() + std::chrono::milliseconds(e->opts.timeout_ms);
@@ -756,10 +828,11 @@ void mt_engine_destroy(mt_engine* e) {
   cudaStreamSynchronize(e->ps);
   cudaStreamSynchronize(e->os);
   for (auto* v : {&e->ready, &e->ready_attn, &e->wd_done, &e->done, &e->g_ready, &e->d2h_done, &e->mlp_done,
-                  &e->timer.ev})
+                  &e->timer.ev, &e->tr_ev})
     for (auto ev : *v)
       if (ev) cudaEventDestroy(ev);
   if (e->fin) cudaEventDestroy(e->fin);
+  if (e->tr_t0) cudaEventDestroy(e->tr_t0);
   for (float* p : e->slab) cudaFreeHost(p);
   delete e;
 }

@@ -280,7 +280,19 @@ typedef struct mt_engine_opts {
   int32_t time_gemms;      /* 1: time every GEMM launch with CUDA events (stats) */
   int32_t no_slab_pool;    /* 1: pin a gradient record per layer and free it after its sink
                               (the "w/o Gradient Slab Pool" ablation of MegaTrain Table 4) */
+  int32_t trace;           /* 1: time every weight upload, layer call and gradient offload of a
+                              step with CUDA events (read back with mt_engine_trace) */
 } mt_engine_opts;
+
+/* One interval of a traced step (MegaTrain Fig. 3's timeline: H2D, compute and
+ * D2H on their three streams). Times are milliseconds on the device clock from
+ * an event recorded on the compute stream when the step starts. */
+typedef struct mt_trace_rec {
+  int32_t kind;     /* 0 weight upload (H2D, prefetch stream), 1 forward, 2 segment re-forward,
+                       3 recompute + backward (compute stream), 4 gradient offload (D2H, offload stream) */
+  int32_t layer;
+  float begin_ms, end_ms;
+} mt_trace_rec;
 
 /* Gradient sink: called on a library thread, in backward order, with layer l's
  * fp32 gradient record (n_elems = record_elems) in a pinned slab. The slab is
@@ -343,6 +355,11 @@ mt_status mt_stream_step_host(mt_engine* e, mt_host_store* store, const mt_bf16*
                               mt_grad_sink sink, void* user);
 
 mt_status mt_engine_stats(const mt_engine* e, mt_stats* out);
+/* The timeline of the engine's last completed step, in issue order (engine
+ * created with trace = 1; call after mt_stream_step returned MT_OK). Writes
+ * min(*n, cap) records to out and the number available to *n.
+ * MT_ERR_INVALID_ARG when tracing is off or no traced step has run. */
+mt_status mt_engine_trace(mt_engine* e, mt_trace_rec* out, int32_t cap, int32_t* n);
 /* Waits (bounded) for the engine's streams and clears a failed step's state. */
 mt_status mt_engine_reset(mt_engine* e);
 void mt_engine_destroy(mt_engine* e);

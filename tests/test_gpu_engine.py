@@ -313,3 +313,33 @@ def test_full_model_step_with_embedding_and_head_hook():
                 assert H.rel(got[k], v) < H.TOL, (l, k)
     finally:
         s.close()
+
+
+def test_traced_step_gives_an_ordered_timeline():
+    """trace = 1: every weight upload, layer call and gradient offload of the last step, in issue
+    order, with the dependencies the engine enforces visible in the times."""
+    s = Stack(TINY, 5, 2, 64, ckpt_interval=2, trace=1)
+    try:
+        with pytest.raises(L.MTError):  # nothing traced before the first step
+            L.mt_engine_trace(s.eng)
+        y0, dx0, g0 = s.step()
+        tl = L.mt_engine_trace(s.eng)
+        kinds = [r["kind"] for r in tl]
+        assert kinds.count("forward") == 5 and kinds.count("backward") == 5 and kinds.count("d2h") == 5
+        assert kinds.count("reforward") == 2  # segments [0,2) and [2,4) are re-run; the last is not
+        assert kinds.count("h2d") >= 5
+        for r in tl:
+            assert -1e-3 <= r["begin_ms"] <= r["end_ms"], r
+        bwd_end = {r["layer"]: r["end_ms"] for r in tl if r["kind"] == "backward"}
+        for r in tl:
+            if r["kind"] == "d2h":  # a layer's last gradient piece leaves after its backward
+                assert r["end_ms"] >= bwd_end[r["layer"]] - 1e-3, r
+        fwd = [r for r in tl if r["kind"] == "forward"]
+        assert [r["layer"] for r in fwd] == list(range(5))
+        assert all(a["end_ms"] <= b["begin_ms"] + 1e-3 for a, b in zip(fwd, fwd[1:]))  # one compute stream
+        # tracing changes no result
+        y1, dx1, g1 = s.step()
+        assert np.array_equal(_as_bits(y0), _as_bits(y1)) and np.array_equal(_as_bits(dx0), _as_bits(dx1))
+        assert all(np.array_equal(g0[k], g1[k]) for k in g0)
+    finally:
+        s.close()

@@ -137,6 +137,9 @@ def test_invalid_arguments_are_rejected_without_a_gpu():
     assert e.value.name == "MT_ERR_UNSUPPORTED"
     opts = L.make_opts(ckpt_interval=0)
     assert L.mt_engine_workspace_bytes(L.make_cfg(**TINY), 2, 1, 8, opts) == 0
+    with pytest.raises(L.MTError) as e:
+        L.mt_engine_trace(None)
+    assert e.value.name == "MT_ERR_INVALID_ARG"
     with pytest.raises(L.MTError) as e:  # the hooked step checks its arguments before any work
         L.mt_stream_step_hooked(None, None, None, None, None, None)
     assert e.value.name == "MT_ERR_INVALID_ARG"

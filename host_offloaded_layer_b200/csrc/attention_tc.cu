@@ -3,8 +3,8 @@
 // accumulators in tensor memory, the operands staged by TMA.
 //
 // Persistent: one CTA per SM walks the (128 query rows, query head, sequence)
-// tiles, longest rows first, so the next tile's Q load and first two S MMAs
-// overlap the current tile's output epilogue.
+// tiles, longest rows first in a snake order, so the next tile's Q load and
+// first two S MMAs overlap the current tile's output epilogue.
 //   warp 0     TMA: lane 0 loads Q per tile and K_j, lane 1 V_j (128 key
 //              rows each), each into its own three-stage ring: a K stage is
 //              free once S_j is done, a V stage once O += P_j V_j is;
@@ -94,6 +94,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// The k-th tile of this CTA in a persistent walk over tiles sorted longest first: round k hands
+// out tiles [k G, k G + G) to the G CTAs in alternating directions (a snake), so the CTA that
+// takes the longest tile of one round takes the shortest of the next and the work stays even.
+__device__ __forceinline__ int snake_tile(int k) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
 // D (+)= A B with A (M = 128 rows in the lanes, 16 bf16 of K packed in pairs
 // along 8 columns) read from tensor memory and B from shared memory.
 __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -177,7 +185,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     if (lane < 2) {
       uint32_t it = 0, tl = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
         const FwdTile w = fwd_tile(t, n_qb, nq, B);
         const int c = (w.h * nkv) / nq;
         const int row0 = w.b * T, q0 = w.qb * BQ;
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     };
     uint32_t it = 0, tl = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+    for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
       const FwdTile w = fwd_tile(t, n_qb, nq, B);
       const int n_kv = min(n_qb, w.qb + 1);
       if (!warp_wait(smem_u32(q_full), tl & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA) || !issue_s(it)) break;
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     const uint32_t col_og = COL_O + g * D;
     uint32_t it = 0, tl = 0, xph = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+    for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
       const FwdTile w = fwd_tile(t, n_qb, nq, B);
       const int q0 = w.qb * BQ, q_row = q0 + r, row0 = w.b * T;
       const int n_kv = min(n_qb, w.qb + 1);
@@ -779,33 +787,48 @@ constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
                           const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
-                          const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int T, int nq,
-                          int nkv, float scale_log2, float scale, int32_t* err) {
+                          const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int B, int T,
+                          int nq, int nkv, float scale_log2, float scale, int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_SMEM_TILES);
-  uint64_t* q_full = bars;         // 1
-  uint64_t* kv_full = bars + 1;    // 5
-  uint64_t* kv_empty = bars + 6;   // 5
-  uint64_t* sp_full = bars + 11;   // 2
-  uint64_t* ds_full = bars + 13;   // 2
-  uint64_t* fin = bars + 15;       // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars;         // 1: Q and dO of the tile loaded
+  uint64_t* q_empty = bars + 1;    // 1: the tile's S / dP MMAs (the readers of Q and dO) are done
+  uint64_t* kv_full = bars + 2;    // 5
+  uint64_t* kv_empty = bars + 7;   // 5
+  uint64_t* sp_full = bars + 12;   // 2
+  uint64_t* ds_full = bars + 14;   // 2
+  uint64_t* dq_full = bars + 16;   // 1: the tile's dQ MMAs are done
+  uint64_t* dq_free = bars + 17;   // 1: the tile's dQ has been read out (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  // query blocks vary slowest, so the launch order is the longest rows first
-  const int qb = gridDim.z - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int c = (h * nkv) / nq;
-  const int q0 = qb * 128;
-  const int n_j = min((T + 63) / 64, (q0 + 128) / 64);
-  const int row0 = b * T;
+  // persistent: tile t is (128 query rows, head, sequence), query blocks from the last (the most
+  // key blocks) down, so the next tile's Q / dO load and first S / dP MMAs overlap this tile's end
+  const int n_qb = (T + 127) / 128;
+  const int n_tiles = n_qb * nq * B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int col_k = (nq + c) * D, col_v = (nq + nkv + c) * D;
+  struct Tile {
+    int qb, h, b, c, q0, n_j, row0;
+  };
+  auto tile = [&](int t) {
+    const int per = nq * B, rest = t % per;
+    Tile w;
+    w.qb = n_qb - 1 - t / per;
+    w.h = rest % nq;
+    w.b = rest / nq;
+    w.c = (w.h * nkv) / nq;
+    w.q0 = w.qb * 128;
+    w.n_j = min((T + 63) / 64, (w.q0 + 128) / 64);
+    w.row0 = w.b * T;
+    return w;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    mbar_init(smem_u32(fin), 1);
+    mbar_init(smem_u32(q_empty), 1);
+    mbar_init(smem_u32(dq_full), 1);
+    mbar_init(smem_u32(dq_free), 8);
     for (int i = 0; i < DQ_KV_STAGES; ++i) {
       mbar_init(smem_u32(&kv_full[i]), 1);
       mbar_init(smem_u32(&kv_empty[i]), 1);
@@ -829,41 +852,51 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      const uint32_t fb = smem_u32(q_full);
-      mbar_expect_tx(fb, 2 * TILE);
-      tma_load_2d(smem_u32(smem + DQ_OFF_Q), &tm_q128, fb, h * D, row0 + q0);
-      tma_load_2d(smem_u32(smem + DQ_OFF_Q + ATOM), &tm_q128, fb, h * D + 64, row0 + q0);
-      tma_load_2d(smem_u32(smem + DQ_OFF_O), &tm_do128, fb, h * D, row0 + q0);
-      tma_load_2d(smem_u32(smem + DQ_OFF_O + ATOM), &tm_do128, fb, h * D + 64, row0 + q0);
-    }
-    __syncwarp();
-    for (int j = 0; j < n_j; ++j) {
-      const int st = j % DQ_KV_STAGES;
-      const uint32_t par = static_cast<uint32_t>(j / DQ_KV_STAGES) & 1u;
-      if (!warp_wait(smem_u32(&kv_empty[st]), par ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+    // ------------------------------------------------------------ TMA producer
+    uint32_t jg = 0, tl = 0;
+    bool ok = true;
+    for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
+      const Tile w = tile(t);
+      const int col_k = (nq + w.c) * D, col_v = (nq + nkv + w.c) * D;
+      if (tl > 0 && !warp_wait(smem_u32(q_empty), (tl - 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
       if (lane == 0) {
-        const uint32_t fb = smem_u32(&kv_full[st]);
-        uint8_t* kt = smem + DQ_OFF_KV + st * 2 * HALF_TILE;
-        uint8_t* vt = kt + HALF_TILE;
-        const int r = row0 + j * 64;
-        mbar_expect_tx(fb, 2 * HALF_TILE);
-        tma_load_2d(smem_u32(kt), &tm_kv64, fb, col_k, r);
-        tma_load_2d(smem_u32(kt + HALF_ATOM), &tm_kv64, fb, col_k + 64, r);
-        tma_load_2d(smem_u32(vt), &tm_kv64, fb, col_v, r);
-        tma_load_2d(smem_u32(vt + HALF_ATOM), &tm_kv64, fb, col_v + 64, r);
+        const uint32_t fb = smem_u32(q_full);
+        mbar_expect_tx(fb, 2 * TILE);
+        tma_load_2d(smem_u32(smem + DQ_OFF_Q), &tm_q128, fb, w.h * D, w.row0 + w.q0);
+        tma_load_2d(smem_u32(smem + DQ_OFF_Q + ATOM), &tm_q128, fb, w.h * D + 64, w.row0 + w.q0);
+        tma_load_2d(smem_u32(smem + DQ_OFF_O), &tm_do128, fb, w.h * D, w.row0 + w.q0);
+        tma_load_2d(smem_u32(smem + DQ_OFF_O + ATOM), &tm_do128, fb, w.h * D + 64, w.row0 + w.q0);
       }
       __syncwarp();
+      for (int j = 0; j < w.n_j; ++j, ++jg) {
+        const int st = jg % DQ_KV_STAGES;
+        const uint32_t par = (jg / DQ_KV_STAGES) & 1u;
+        if (!warp_wait(smem_u32(&kv_empty[st]), par ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&kv_full[st]);
+          uint8_t* kt = smem + DQ_OFF_KV + st * 2 * HALF_TILE;
+          uint8_t* vt = kt + HALF_TILE;
+          const int r = w.row0 + j * 64;
+          mbar_expect_tx(fb, 2 * HALF_TILE);
+          tma_load_2d(smem_u32(kt), &tm_kv64, fb, col_k, r);
+          tma_load_2d(smem_u32(kt + HALF_ATOM), &tm_kv64, fb, col_k + 64, r);
+          tma_load_2d(smem_u32(vt), &tm_kv64, fb, col_v, r);
+          tma_load_2d(smem_u32(vt + HALF_ATOM), &tm_kv64, fb, col_v + 64, r);
+        }
+        __syncwarp();
+      }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_sp = idesc_bf16(128, 64, false, false);  // S = Q K^T, dP = dO V^T
     constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);    // dQ += dS K (K is MN-major)
     const uint32_t q_base = smem_u32(smem + DQ_OFF_Q), o_base = smem_u32(smem + DQ_OFF_O);
-    bool ok = warp_wait(smem_u32(q_full), 0, abort_flag, err, DEV_ERR_TIMEOUT_MMA);
-    auto issue_sp = [&](int j) -> bool {
-      const int st = j & 1, sk = j % DQ_KV_STAGES;
-      if (!warp_wait(smem_u32(&kv_full[sk]), static_cast<uint32_t>(j / DQ_KV_STAGES) & 1u, abort_flag, err,
-                     DEV_ERR_TIMEOUT_MMA))
+    auto issue_sp = [&](uint32_t i) -> bool {
+      const int st = i & 1, sk = i % DQ_KV_STAGES;
+      if (!warp_wait(smem_u32(&kv_full[sk]), (i / DQ_KV_STAGES) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA))
         return false;
       fence_after();
       if (lane == 0) {
@@ -883,81 +916,106 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       __syncwarp();
       return true;
     };
-    if (ok) ok = issue_sp(0);
-    for (int j = 0; j < n_j && ok; ++j) {
-      const int st = j & 1;
-      if (j + 1 < n_j && !issue_sp(j + 1)) {
-        ok = false;
-        break;
-      }
-      if (!warp_wait(smem_u32(&ds_full[st]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      if (lane == 0) {
-        const int sk = j % DQ_KV_STAGES;
-        const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + sk * 2 * HALF_TILE);
-#pragma unroll
-        for (int kk = 0; kk < 64 / 16; ++kk) {
-          // key columns [16 kk, 16 kk + 16): group kk / 2's packed columns, second half at + 8
-          const uint32_t a_col = static_cast<uint32_t>(st * 64 + (kk >> 1) * 32 + (kk & 1) * 8);
-          umma_bf16_tmem_a(tmem + DQ_COL_DQ, tmem + DQ_COL_S + a_col, smem_desc(k_base + kk * 2048, HALF_ATOM, 1024),
-                           idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+    uint32_t jg = 0, tl = 0;
+    bool ok = true;
+    for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
+      const Tile w = tile(t);
+      if (!warp_wait(smem_u32(q_full), tl & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA) || !issue_sp(jg)) break;
+      for (int j = 0; j < w.n_j && ok; ++j) {
+        const uint32_t i = jg + j;
+        const int st = i & 1;
+        if (j + 1 < w.n_j) {
+          if (!issue_sp(i + 1)) {
+            ok = false;
+            break;
+          }
+        } else {
+          if (lane == 0) umma_commit(smem_u32(q_empty));  // every S / dP MMA of the tile is issued
+          __syncwarp();
         }
-        umma_commit(smem_u32(&kv_empty[sk]));
+        if (!warp_wait(smem_u32(&ds_full[st]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        // the first dQ MMA of a tile overwrites dQ: the previous tile's must have been read out
+        if (j == 0 && tl > 0 && !warp_wait(smem_u32(dq_free), (tl - 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        if (lane == 0) {
+          const int sk = i % DQ_KV_STAGES;
+          const uint32_t k_base = smem_u32(smem + DQ_OFF_KV + sk * 2 * HALF_TILE);
+#pragma unroll
+          for (int kk = 0; kk < 64 / 16; ++kk) {
+            // key columns [16 kk, 16 kk + 16): group kk / 2's packed columns, second half at + 8
+            const uint32_t a_col = static_cast<uint32_t>(st * 64 + (kk >> 1) * 32 + (kk & 1) * 8);
+            umma_bf16_tmem_a(tmem + DQ_COL_DQ, tmem + DQ_COL_S + a_col,
+                             smem_desc(k_base + kk * 2048, HALF_ATOM, 1024), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&kv_empty[sk]));
+        }
+        __syncwarp();
       }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(dq_full));
       __syncwarp();
+      jg += w.n_j;
     }
-    if (lane == 0) umma_commit(smem_u32(fin));
-    __syncwarp();
   } else {
+    // ------------------------------------------------------------ dS, one thread per query row and group
     const int g = (warp - 2) >> 2;  // key columns [32 g, 32 g + 32) of each 64-column block
     const int qw = warp & 3;
     const int r = qw * 32 + lane;
-    const int q_row = q0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
-    const int64_t sb = (static_cast<int64_t>(b) * nq + h) * T;
-    const float lse2 = q_row < T ? lse[sb + q_row] * LOG2E : 0.f;
-    const float dl = q_row < T ? delta[sb + q_row] : 0.f;
+    uint32_t jg = 0, tl = 0;
     bool ok = true;
-    for (int j = 0; j < n_j; ++j) {
-      const int st = j & 1;
-      if (!warp_wait(smem_u32(&sp_full[st]), (j >> 1) & 1, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
-        ok = false;
-        break;
+    for (int t = snake_tile(0), k = 0; t < n_tiles && ok; t = snake_tile(++k), ++tl) {
+      const Tile w = tile(t);
+      const int q_row = w.q0 + r;
+      const int64_t sb = (static_cast<int64_t>(w.b) * nq + w.h) * T;
+      const float lse2 = q_row < T ? lse[sb + q_row] * LOG2E : 0.f;
+      const float dl = q_row < T ? delta[sb + q_row] : 0.f;
+      for (int j = 0; j < w.n_j; ++j) {
+        const uint32_t i = jg + j;
+        const int st = i & 1;
+        if (!warp_wait(smem_u32(&sp_full[st]), (i >> 1) & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        float sv[32], dv[32];
+        {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, u);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
+          tmem_ld32(tmem + lane_base + DQ_COL_DP + st * 64 + g * 32, u);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
+        }
+        const int k0 = j * 64 + g * 32;
+        const bool diag = k0 + 31 > w.q0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float p = ex2(fmaf(sv[e], scale_log2, -lse2));
+          if (diag && k0 + e > q_row) p = 0.f;
+          dv[e] = p * (dv[e] - dl);
+        }
+        {  // dS over the S values just read
+          uint32_t pd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pd[e] = pack_bf16(dv[2 * e], dv[2 * e + 1]);
+          tmem_st16(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, pd);
+        }
+        fence_before();
+        warp_arrive(smem_u32(&ds_full[st]));
       }
+      if (!ok) break;
+      jg += w.n_j;
+      if (!warp_wait(smem_u32(dq_full), tl & 1u, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
-      float sv[32], dv[32];
-      {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
-        tmem_ld32(tmem + lane_base + DQ_COL_DP + st * 64 + g * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dv[e] = __uint_as_float(u[e]);
-      }
-      const int k0 = j * 64 + g * 32;
-      const bool diag = k0 + 31 > q0;
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float p = ex2(fmaf(sv[e], scale_log2, -lse2));
-        if (diag && k0 + e > q_row) p = 0.f;
-        dv[e] = p * (dv[e] - dl);
-      }
-      {  // dS over the S values just read
-        uint32_t pd[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) pd[e] = pack_bf16(dv[2 * e], dv[2 * e + 1]);
-        tmem_st16(tmem + lane_base + DQ_COL_S + st * 64 + g * 32, pd);
-      }
-      fence_before();
-      warp_arrive(smem_u32(&ds_full[st]));
-    }
-    if (ok && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
-      fence_after();
-      __nv_bfloat16* out = dqkv + (static_cast<int64_t>(row0) + q_row) * ld + static_cast<int64_t>(h) * D + g * 64;
+      __nv_bfloat16* out = dqkv + (static_cast<int64_t>(w.row0) + q_row) * ld + static_cast<int64_t>(w.h) * D + g * 64;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {  // group g writes dQ columns [64 g, 64 g + 64)
         uint32_t u[32];
@@ -965,15 +1023,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (q_row < T) {
 #pragma unroll
           for (int qd = 0; qd < 4; ++qd) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(u[qd * 8 + 0]) * scale, __uint_as_float(u[qd * 8 + 1]) * scale);
-            w.y = pack_bf16(__uint_as_float(u[qd * 8 + 2]) * scale, __uint_as_float(u[qd * 8 + 3]) * scale);
-            w.z = pack_bf16(__uint_as_float(u[qd * 8 + 4]) * scale, __uint_as_float(u[qd * 8 + 5]) * scale);
-            w.w = pack_bf16(__uint_as_float(u[qd * 8 + 6]) * scale, __uint_as_float(u[qd * 8 + 7]) * scale);
-            *reinterpret_cast<uint4*>(out + ch * 32 + qd * 8) = w;
+            uint4 wv;
+            wv.x = pack_bf16(__uint_as_float(u[qd * 8 + 0]) * scale, __uint_as_float(u[qd * 8 + 1]) * scale);
+            wv.y = pack_bf16(__uint_as_float(u[qd * 8 + 2]) * scale, __uint_as_float(u[qd * 8 + 3]) * scale);
+            wv.z = pack_bf16(__uint_as_float(u[qd * 8 + 4]) * scale, __uint_as_float(u[qd * 8 + 5]) * scale);
+            wv.w = pack_bf16(__uint_as_float(u[qd * 8 + 6]) * scale, __uint_as_float(u[qd * 8 + 7]) * scale);
+            *reinterpret_cast<uint4*>(out + ch * 32 + qd * 8) = wv;
           }
         }
       }
+      fence_before();
+      warp_arrive(smem_u32(dq_free));
     }
   }
 
@@ -1012,8 +1072,9 @@ mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o,
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
   const float scale_log2 = LOG2E * scale;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(dqkv);
-  dim3 gq(nq, B, (T + 127) / 128);
-  attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, T, nq, nkv,
+  const int64_t dq_tiles = static_cast<int64_t>((T + 127) / 128) * nq * B;
+  const int gq = static_cast<int>(std::min<int64_t>(dq_tiles, num_sms()));
+  attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, B, T, nq, nkv,
                                                                 scale_log2, scale, err);
   MT_TRY(launch_check("attn_bwd_dq_tc_kernel"));
   dim3 gk(nkv, B, (T + 127) / 128);

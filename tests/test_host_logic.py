@@ -209,3 +209,30 @@ def test_embedding_sort_is_stable_and_complete():
     assert list(order) == [3, 1, 5, 0, 2, 4]
     with pytest.raises(L.MTError):
         L.mt_embed_sort(np.array([4], np.int32), 1, 4, order, start)
+
+
+def test_gemm_traffic_is_tied_to_the_gemm_code_not_its_comments(tmp_path, monkeypatch):
+    """bench.py reports the committed GEMM DRAM traffic only for the code it was measured on:
+    the hash ignores // comments and blank lines, and any code change (or another workload)
+    turns the figure into null."""
+    import importlib
+    import shutil
+    import sys
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    csrc = tmp_path / "host_offloaded_layer_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    for f in ("gemm.cu", "tcgen05.cuh"):
+        shutil.copy(os.path.join(ROOT, "host_offloaded_layer_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.gemm_source_hash()
+    (tmp_path / "profiles" / "gemm2_kernel_traffic.txt").write_text(
+        "# header: with a colon\nkernel_code_sha256: %s\nworkload: w\ndram_bytes_per_launch: 123\n" % h)
+    assert bench.gemm_traffic("w") == 123.0
+    assert bench.gemm_traffic("other") is None
+    g = csrc / "gemm.cu"
+    g.write_text(g.read_text() + "\n// a comment only\n\n")
+    assert bench.gemm_source_hash() == h and bench.gemm_traffic("w") == 123.0
+    g.write_text(g.read_text() + "static int changed_code = 1;\n")
+    assert bench.gemm_source_hash() != h and bench.gemm_traffic("w") is None

@@ -303,7 +303,7 @@ typedef struct mt_engine mt_engine;
 
 typedef struct mt_stats {
   double step_ms;             /* host wall time of the last step */
-  double h2d_ms, d2h_ms;      /* device time of the copies (sum over copies) */
+  double h2d_ms, d2h_ms;      /* reserved, 0 (per-copy device times: mt_engine_trace) */
   uint64_t h2d_bytes, d2h_bytes;
   uint64_t layer_fwd_calls, layer_bwd_calls, weight_loads;
   double exec_flops;          /* FLOPs the kernels executed in the last step */
@@ -354,6 +354,8 @@ mt_status mt_stream_step_host(mt_engine* e, mt_host_store* store, const mt_bf16*
                               const mt_bf16* dy_top_host, mt_bf16* y_top_host, mt_bf16* dx0_host,
                               mt_grad_sink sink, void* user);
 
+/* Counters of the engine's last step (mt_stats above; h2d_ms and d2h_ms stay 0: the copies are
+ * timed by the trace below). MT_ERR_INVALID_ARG on NULL. */
 mt_status mt_engine_stats(const mt_engine* e, mt_stats* out);
 /* The timeline of the engine's last completed step, in issue order (engine
  * created with trace = 1; call after mt_stream_step returned MT_OK). Writes

@@ -631,17 +631,6 @@ mt_status fwd_t(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float*
   return MT_OK;
 }
 
-// head_dim 128 runs the tcgen05 backward unless MT_ATTN_BWD=mma is set (kept for
-// comparison measurements).
-bool use_tc_bwd() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MT_ATTN_BWD");
-    v = (e && std::string(e) == "mma") ? 0 : 1;
-  }
-  return v == 1;
-}
-
 template <int D>
 mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16* d_o, int64_t ld_o, const float* lse,
                 mt_bf16* dqkv, int B, int T, int nq, int nkv, float* delta, cudaStream_t st) {
@@ -658,7 +647,9 @@ mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16*
   attn_delta_kernel<D><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, delta, rows, T, nq);
   MT_TRY(launch_check("attn_delta_kernel"));
-  if (D == 128 && use_tc_bwd()) return attn_bwd_tc_launch(qkv, ld, d_o, ld_o, lse, delta, dqkv, B, T, nq, nkv, st);
+  if constexpr (D == 128) {
+    return attn_bwd_tc_launch(qkv, ld, d_o, ld_o, lse, delta, dqkv, B, T, nq, nkv, st);
+  } else {
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
   const float scale_log2 = LOG2E * scale;
   dim3 gq((T + C::BQ - 1) / C::BQ, nq, B);
@@ -676,6 +667,7 @@ mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16*
   // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)
   add_exec_flops(14.0 * B * nq * D * (0.5 * double(T) * double(T)));
   return MT_OK;
+  }
 }
 
 }  // namespace
@@ -687,22 +679,11 @@ uint64_t attn_bwd_ws_bytes(int B, int T, int nq) {
 mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T,
                              int nq, int nkv, cudaStream_t st);
 
-// head_dim 128 runs the tcgen05 forward unless MT_ATTN_FWD=mma is set (kept for
-// comparison measurements); head_dim 64 runs the mma.sync forward.
-static bool use_tc_fwd() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MT_ATTN_FWD");
-    v = (e && std::string(e) == "mma") ? 0 : 1;
-  }
-  return v == 1;
-}
-
+// head_dim 128 runs the tcgen05 forward, head_dim 64 the mma.sync one.
 mt_status attn_fwd_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float* lse, int B, int T, int nq,
                           int nkv, int d, cudaStream_t st) {
   if (B == 0 || T == 0) return MT_OK;
-  if (d == 128 && use_tc_fwd()) return attn_fwd_tc_launch(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
-  if (d == 128) return fwd_t<128>(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
+  if (d == 128) return attn_fwd_tc_launch(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
   if (d == 64) return fwd_t<64>(qkv, ld, o, ld_o, lse, B, T, nq, nkv, st);
   return fail(MT_ERR_UNSUPPORTED, "attention supports head_dim 64 and 128, not %d", d);
 }

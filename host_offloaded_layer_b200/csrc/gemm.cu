@@ -8,17 +8,19 @@
 // the MegaTrain pages ("stateless layer templates", abstract) runs for every
 // streamed layer.
 //
-// Design
-// - Tile 128 x 256 x 64 (bf16), 4-stage shared-memory ring, one CTA per SM,
-//   persistent over output tiles (grouped raster, 16 row-blocks per group).
-// - Warp 0: TMA producer. Warp 1: TMEM allocation and the MMA issuer.
-//   Warps 2-5: epilogue (tcgen05.ld of the fp32 accumulator, bias/residual,
-//   bf16 or fp32 store).
-// - Two 256-column accumulators in TMEM (512 columns): the epilogue of one
-//   tile overlaps the main loop of the next.
-// - Operands are staged with 128-byte swizzle. K-major tiles are one TMA box
-//   of 64 (K) x rows; MN-major tiles are boxes of 64 (M or N) x 64 (K) placed
-//   8 KiB apart, which is the descriptor's leading-byte offset.
+// Design (details at the 2-SM kernel below)
+// - A cluster of two CTAs on two SMs computes a 256 x 256 output tile with
+//   tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), persistent over the
+//   output tiles; the weight-gradient layout at K >= 8192 uses a 256 x 512 tile.
+// - Per CTA: warp 0 is the TMA producer, warp 1 allocates TMEM and (in the
+//   even CTA) issues the MMAs for the pair, the remaining warps run the
+//   epilogue (tcgen05.ld of the fp32 accumulator; bias, residual, fp32
+//   accumulate, SwiGLU forward or backward; bf16 or fp32 stores).
+// - Two 256-column accumulators in TMEM: the epilogue of one tile overlaps
+//   the main loop of the next.
+// - Operands are staged with 128-byte swizzle. K-major tiles are boxes of
+//   64 (K) x 128 rows; MN-major tiles are boxes of 64 (M or N) x 64 (K) placed
+//   one atom apart, which is the descriptor's leading-byte offset.
 // - Every mbarrier wait is bounded (4 s); when one runs out the kernel sets
 //   the device error word and all roles leave their loops, free TMEM and exit.
 #include <cuda.h>
@@ -38,14 +40,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_TILE = BM * BK * 2;  // 16 KiB
-constexpr int B_TILE = BN * BK * 2;  // 32 KiB
-constexpr int MN_BOX = 64 * BK * 2;  // one 64 x 64 MN-major box: 8 KiB
-constexpr int SMEM_TILES = STAGES * (A_TILE + B_TILE);
-constexpr int NUM_THREADS = 192;
+constexpr int MN_BOX = 64 * 64 * 2;  // one 64 x 64 MN-major box: 8 KiB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int SMEM_BYTES = SMEM_TILES + 256 + 1024;
 
 struct EpiArgs {
   void* C;
@@ -66,13 +62,6 @@ struct EpiArgs {
   __nv_bfloat16* gu;
   int64_t ld_gu;
 };
-
-// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and
-// B bf16 (bits 7-9 and 10-12 = 1), A/B major bits 15/16, N>>3 at 17, M>>4 at 24.
-__host__ __device__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-         (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-}
 
 // Output-tile order. raster 0: groups of 16 row-blocks, columns within a
 // group; raster 1: row-major over all column blocks (the B operand stays in
@@ -273,184 +262,11 @@ __device__ __forceinline__ void store_swiglu(const EpiArgs& ep, int row, int f0,
   }
 }
 
-template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, EpiArgs ep,
-                int32_t* err) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
-  uint64_t* full = bars;                // TMA -> MMA, one per stage
-  uint64_t* empty = bars + STAGES;      // MMA -> TMA, one per stage
-  uint64_t* tfull = bars + 2 * STAGES;  // MMA -> epilogue, one per accumulator
-  uint64_t* tempty = tfull + 2;         // epilogue -> MMA, one per accumulator
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_m = (ep.M + BM - 1) / BM, num_n = (ep.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
-  const int num_kb = (ep.K + BK - 1) / BK;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 128);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
-      const int m0 = mb * BM, n0 = nb * BN;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        if (!warp_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_PRODUCER)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          const uint32_t fb = smem_u32(&full[s]);
-          const uint32_t a_dst = smem_u32(sA + s * A_TILE), b_dst = smem_u32(sB + s * B_TILE);
-          const int k0 = kb * BK;
-          // Boxes that lie wholly past M or N are skipped: those rows of the
-          // tile only feed output rows/columns that are never stored.
-          uint32_t bytes = 0;
-          if (!A_MN) {
-            bytes += A_TILE;
-          } else {
-            for (int j = 0; j < BM / 64; ++j)
-              if (m0 + 64 * j < ep.M) bytes += MN_BOX;
-          }
-          if (!B_MN) {
-            bytes += B_TILE;
-          } else {
-            for (int j = 0; j < BN / 64; ++j)
-              if (n0 + 64 * j < ep.N) bytes += MN_BOX;
-          }
-          mbar_expect_tx(fb, bytes);
-          if (!A_MN) {
-            tma_load_2d(a_dst, &tmA, fb, k0, m0);
-          } else {
-            for (int j = 0; j < BM / 64; ++j)
-              if (m0 + 64 * j < ep.M) tma_load_2d(a_dst + j * MN_BOX, &tmA, fb, m0 + 64 * j, k0);
-          }
-          if (!B_MN) {
-            tma_load_2d(b_dst, &tmB, fb, k0, n0);
-          } else {
-            for (int j = 0; j < BN / 64; ++j)
-              if (n0 + 64 * j < ep.N) tma_load_2d(b_dst + j * MN_BOX, &tmB, fb, n0 + 64 * j, k0);
-          }
-        }
-        __syncwarp();
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = make_idesc(A_MN, B_MN);
-    uint32_t it = 0;
-    int tl = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tl) {
-      const int ab = tl & 1;
-      const uint32_t aph = (tl >> 1) & 1u;
-      if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
-      fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        if (!warp_wait(smem_u32(&full[s]), ph, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) {
-          ok = false;
-          break;
-        }
-        fence_after();
-        if (lane == 0) {
-          const uint32_t a_base = smem_u32(sA + s * A_TILE), b_base = smem_u32(sB + s * B_TILE);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            // K-major: advance 16 elements (32 bytes) inside the swizzled row.
-            // MN-major: advance 16 K-rows (two 8-row groups of 1 KiB).
-            const uint64_t ad = A_MN ? smem_desc(a_base + kk * 2048, MN_BOX, 1024) : smem_desc(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc(b_base + kk * 2048, MN_BOX, 1024) : smem_desc(b_base + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(smem_u32(&empty[s]));
-        }
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (lane == 0) umma_commit(smem_u32(&tfull[ab]));
-      __syncwarp();
-    }
-  } else {
-    // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are readable by this warp
-    int tl = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
-      const int ab = tl & 1;
-      const uint32_t aph = (tl >> 1) & 1u;
-      int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
-      if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
-      fence_after();
-      const int row = mb * BM + q * 32 + lane;
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = nb * BN + c * 32;
-        if (col0 >= ep.N) break;  // uniform across the warp
-        uint32_t r[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN + c * 32), r);
-        if (row < ep.M) {
-          if (ep.swiglu == 2)
-            store_swiglu_bwd(ep, row, col0, r);
-          else
-            store_chunk(ep, row, col0, r);
-        }
-      }
-      fence_before();
-      mbar_arrive(smem_u32(&tempty[ab]));
-    }
-  }
-
-  fence_before();
-  __syncthreads();
-  fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
-  }
-}
-
 // ============================================================== 2-SM kernel
-// The same contraction with tcgen05.mma.cta_group::2: a cluster of two CTAs
-// on two SMs computes a 256 x 256 output tile. Each CTA stages its own 128
-// rows of A and its own 128 columns' worth of B (6 stages of 32 KiB), so per
-// FLOP each SM moves a third less operand data through shared memory than the
-// one-SM 128 x 256 tile. The even CTA issues the MMAs for the pair; its full
+// tcgen05.mma.cta_group::2: a cluster of two CTAs on two SMs computes a
+// 256 x 256 output tile. Each CTA stages its own 128 rows of A and its own 128
+// columns' worth of B (3 stages of 64 KiB), so per FLOP each SM moves a third
+// less operand data through shared memory than a one-SM 128 x 256 tile. The even CTA issues the MMAs for the pair; its full
 // barriers count both CTAs' TMA bytes, each MMA commit signals both CTAs'
 // empty / accumulator-full barriers, and both CTAs' epilogue warps arrive on
 // the even CTA's accumulator-empty barrier. Every CTA loads its own operands
@@ -782,22 +598,6 @@ mt_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return MT_OK;
 }
 
-template <bool A_MN, bool B_MN>
-mt_status launch_1sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return fail(MT_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(attr_err));
-  const int num_tiles = ((ep.M + BM - 1) / BM) * ((ep.N + BN - 1) / BN);
-  const int grid = std::min(num_tiles, num_sms());
-  int32_t* err = device_error_word();
-  if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
-  gemm_kernel<A_MN, B_MN><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, ep, err);
-  return launch_check("gemm_kernel");
-}
-
 // Largest number of 2-CTA clusters of gemm2_kernel that fit on the device at once.
 template <bool A_MN, bool B_MN, int KA, int NH>
 int max_pair_clusters() {
@@ -839,51 +639,18 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
   return launch_check("gemm2_kernel");
 }
 
-// K atoms per stage of the 2-SM kernel: 2 (3 stages of 128) unless
-// MT_GEMM_KATOMS=1 (6 stages of 64) is set. Eight MMAs per barrier round trip
-// measured 7-16% faster than four on every layout of the layer.
-int gemm_katoms() {
-  static int v = 0;
-  if (v == 0) {
-    const char* e = getenv("MT_GEMM_KATOMS");
-    v = (e && std::string(e) == "1") ? 1 : 2;
-  }
-  return v;
-}
-
 // Pair-tile width. The 256 x 512 tile (NH = 2) measured 4-7% faster on the
 // weight-gradient layout (both operands MN-major, K = tokens >= 16384, fp32 out),
 // where a tile's main loop is long enough to hide its unbuffered epilogue, and
 // 2-5% slower on the forward and input-gradient shapes of the layer (K = 3584):
-// it is used for the weight-gradient layout with K >= 8192. MT_GEMM_WIDE=1 / 0
-// forces it on / off (comparison measurements).
-int gemm_wide_mode() {
-  static int v = -2;
-  if (v == -2) {
-    const char* e = getenv("MT_GEMM_WIDE");
-    v = !e ? -1 : (std::string(e) == "1" ? 1 : 0);
-  }
-  return v;
-}
-
+// it is used for the weight-gradient layout with K >= 8192. Every other launch
+// runs the 256 x 256 tile with three stages of 128-wide K (eight MMAs per
+// barrier round trip measured 7-16% faster than four on every layout).
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
-  const int mode = gemm_wide_mode();
-  const bool wide = mode == 1 || (mode == -1 && A_MN && B_MN && ep.swiglu == 0 && ep.K >= 8192);
+  const bool wide = A_MN && B_MN && ep.swiglu == 0 && ep.K >= 8192;
   if (wide) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
-  return gemm_katoms() == 2 ? launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st)
-                            : launch_2sm_ka<A_MN, B_MN, 1, 1>(ta, tb, ep, st);
-}
-
-// Which kernel runs: the 2-SM kernel unless MT_GEMM_KERNEL=1sm is set (kept for
-// comparison measurements).
-bool use_2sm() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MT_GEMM_KERNEL");
-    v = (e && std::string(e) == "1sm") ? 0 : 1;
-  }
-  return v == 1;
+  return launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st);
 }
 
 // Tile order that keeps the smaller operand resident in L2 when it fits.
@@ -904,15 +671,13 @@ mt_status gemm_dispatch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16*
                         EpiArgs ep, cudaStream_t st) {
   const int64_t M = ep.M, N = ep.N, K = ep.K;
   if (M == 0 || N == 0) return MT_OK;
-  const bool two = use_2sm();
-  const uint32_t b_rows = two ? 128 : BN;  // rows of a K-major B box
   CUtensorMap ta, tb;
   if (!a_mn)
     MT_TRY(make_map(&ta, A, K, M, lda, 64, 128));
   else
     MT_TRY(make_map(&ta, A, M, K, lda, 64, 64));
   if (!b_mn)
-    MT_TRY(make_map(&tb, B, K, N, ldb, 64, b_rows));
+    MT_TRY(make_map(&tb, B, K, N, ldb, 64, 128));
   else
     MT_TRY(make_map(&tb, B, N, K, ldb, 64, 64));
   ep.raster = pick_raster(M, N, K);
@@ -920,25 +685,14 @@ mt_status gemm_dispatch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16*
   GemmTimer* tm = current_gemm_timer();
   if (tm) tm->before(st);
   mt_status s;
-  if (two) {
-    if (!a_mn && !b_mn)
-      s = launch_2sm<false, false>(ta, tb, ep, st);
-    else if (!a_mn && b_mn)
-      s = launch_2sm<false, true>(ta, tb, ep, st);
-    else if (a_mn && !b_mn)
-      s = launch_2sm<true, false>(ta, tb, ep, st);
-    else
-      s = launch_2sm<true, true>(ta, tb, ep, st);
-  } else {
-    if (!a_mn && !b_mn)
-      s = launch_1sm<false, false>(ta, tb, ep, st);
-    else if (!a_mn && b_mn)
-      s = launch_1sm<false, true>(ta, tb, ep, st);
-    else if (a_mn && !b_mn)
-      s = launch_1sm<true, false>(ta, tb, ep, st);
-    else
-      s = launch_1sm<true, true>(ta, tb, ep, st);
-  }
+  if (!a_mn && !b_mn)
+    s = launch_2sm<false, false>(ta, tb, ep, st);
+  else if (!a_mn && b_mn)
+    s = launch_2sm<false, true>(ta, tb, ep, st);
+  else if (a_mn && !b_mn)
+    s = launch_2sm<true, false>(ta, tb, ep, st);
+  else
+    s = launch_2sm<true, true>(ta, tb, ep, st);
   if (tm) tm->after(st, flops);
   add_exec_flops(flops);
   return s;
@@ -995,12 +749,9 @@ mt_status tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
   return make_map(m, ptr, inner, outer, ld_elems, box_inner, box_outer);
 }
 
-bool gemm_swiglu_available() { return use_2sm(); }
-
 mt_status gemm_swiglu_launch(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m, int64_t ldm,
                              mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st) {
   if (M == 0 || F == 0) return MT_OK;
-  if (!use_2sm()) return fail(MT_ERR_UNSUPPORTED, "the fused SwiGLU epilogue needs the 2-SM GEMM kernel");
   CUtensorMap ta, tb;
   MT_TRY(make_map(&ta, A, K, M, lda, 64, 128));
   MT_TRY(make_map(&tb, Wgu, K, 2 * F, ldw, 64, 128));

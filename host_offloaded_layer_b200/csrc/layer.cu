@@ -29,21 +29,7 @@ mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, i
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
 mt_status rope_launch(mt_bf16*, int64_t, int, int, int, int, float, bool, cudaStream_t);
-mt_status swiglu_bwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, int64_t, int, cudaStream_t);
 
-// The SwiGLU backward runs in the epilogue of the dm GEMM unless
-// MT_SWIGLU_BWD=split selects the GEMM plus the stand-alone kernel (kept for
-// comparison measurements).
-bool swiglu_bwd_fused() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MT_SWIGLU_BWD");
-    v = (e && std::string(e) == "split") ? 0 : 1;
-  }
-  return v == 1;
-}
-
-mt_status swiglu_fwd_launch(const mt_bf16*, mt_bf16*, int64_t, int, cudaStream_t);
 mt_status colsum_launch(const mt_bf16*, const mt_bf16*, const float*, int64_t, int64_t, int64_t, float*, void*,
                         cudaStream_t);
 uint64_t colsum_ws_bytes(int64_t rows, int64_t cols);
@@ -51,7 +37,6 @@ mt_status attn_fwd_launch(const mt_bf16*, int64_t, mt_bf16*, int64_t, float*, in
 mt_status attn_bwd_launch(const mt_bf16*, int64_t, const mt_bf16*, const mt_bf16*, int64_t, const float*, mt_bf16*,
                           int, int, int, int, int, void*, cudaStream_t);
 uint64_t attn_bwd_ws_bytes(int B, int T, int nq);
-bool gemm_swiglu_available();
 mt_status gemm_swiglu_launch(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m, int64_t ldm,
                              mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st);
 
@@ -116,19 +101,14 @@ mt_status attention_half(const Geom& G, const mt_bf16* w, const mt_bf16* x, int 
   return MT_OK;
 }
 
-// [g|u] = h2c Wgu^T; m = silu(g) * u for one chunk of rows. With the 2-SM GEMM
-// the SwiGLU is its epilogue (m from the fp32 accumulators; g and u are only
-// written when the backward needs them); otherwise a separate pass.
+// [g|u] = h2c Wgu^T; m = silu(g) * u for one chunk of rows, the SwiGLU in the
+// GEMM's epilogue (m from the fp32 accumulators; g and u are only written when
+// the backward needs them).
 mt_status mlp_up(const Geom& G, const mt_bf16* w, const mt_bf16* h2c, int64_t rows, const LayerWs& ws, bool need_gu,
                  cudaStream_t st) {
   const mt_param_offsets& O = G.off;
-  if (gemm_swiglu_available())
-    return gemm_swiglu_launch(h2c, G.H, w + O.wg, G.H, ws.m, G.F, need_gu ? ws.gu : nullptr, 2 * G.F, rows, G.F, G.H,
-                              st);
-  MT_TRY(gemm_launch(h2c, G.H, false, w + O.wg, G.H, false, ws.gu, 2 * G.F, false, false, rows, 2 * G.F, G.H, nullptr,
-                     nullptr, 0, st));
-  MT_TRY(swiglu_fwd_launch(ws.gu, ws.m, rows, static_cast<int>(G.F), st));
-  return MT_OK;
+  return gemm_swiglu_launch(h2c, G.H, w + O.wg, G.H, ws.m, G.F, need_gu ? ws.gu : nullptr, 2 * G.F, rows, G.F, G.H,
+                            st);
 }
 
 }  // namespace
@@ -234,15 +214,8 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
     MT_TRY(gemm_launch(dyc, G.H, true, w.m, G.F, true, dw_dev + O.wd, G.F, true, acc, G.H, G.F, rows, nullptr, nullptr,
                        0, st));
     if (wd_done && r0 + rows >= M) MT_CUDA(cudaEventRecord(wd_done, st));  // dWd is final after the last chunk
-    if (swiglu_bwd_fused()) {
-      // dm = dy Wd, and in the same GEMM's epilogue [dg|du] in place over [g|u]
-      MT_TRY(gemm_swiglu_bwd_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.gu, 2 * G.F, rows, G.F, G.H, st));
-    } else {
-      // dm = dy Wd (into the m buffer), then [dg|du] in place over [g|u]
-      MT_TRY(gemm_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.m, G.F, false, false, rows, G.F, G.H, nullptr,
-                         nullptr, 0, st));
-      MT_TRY(swiglu_bwd_launch(w.m, w.gu, w.gu, rows, static_cast<int>(G.F), st));
-    }
+    // dm = dy Wd, and in the same GEMM's epilogue [dg|du] in place over [g|u]
+    MT_TRY(gemm_swiglu_bwd_launch(dyc, G.H, false, w_dev + O.wd, G.F, true, w.gu, 2 * G.F, rows, G.F, G.H, st));
     // dWgu (+)= dgu^T h2
     MT_TRY(gemm_launch(w.gu, 2 * G.F, true, h2c, G.H, true, dw_dev + O.wg, G.H, true, acc, 2 * G.F, G.H, rows, nullptr,
                        nullptr, 0, st));

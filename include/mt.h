@@ -151,8 +151,7 @@ mt_status mt_gemm_bf16(const mt_bf16* A, int64_t lda, int32_t a_mn_major,
  * K-major. m[r, j] = silu(g) * u with g = A_r . Wg_j and u = A_r . Wu_j taken
  * from the fp32 accumulators; when gu is not NULL, g and u are also stored
  * (bf16) to gu[r, j] and gu[r, F + j]. Pointers 16-byte aligned; lda, ldw,
- * ldm, ld_gu and F multiples of 8. MT_ERR_UNSUPPORTED when the library runs
- * its one-SM GEMM kernel (MT_GEMM_KERNEL=1sm). */
+ * ldm, ld_gu and F multiples of 8. */
 mt_status mt_gemm_swiglu_bf16(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m,
                               int64_t ldm, mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, void* stream);
 

@@ -9,8 +9,9 @@ store and its fp32 gradients streamed out through the slab pool. Workloads
 (synthetic data, seeded, N(0, 0.02) weights, N(0, 1) inputs and dY):
 
   1 tiny      hidden 256, 4/2 heads x 64, FFN 688, 1 layer, batch 2 x 128
-  2 7b_x4     Qwen2.5-7B layer shape x 4 layers, batch 8 x 1024, K = 4  (default)
-  3 7b_x28    7B shape x 28 layers, batch 96 x 1024, K = 4
+  2 7b_x4     Qwen2.5-7B layer shape x 4 layers, batch 8 x 1024, K = 4
+  3 7b_x28    7B shape x 28 layers, batch 96 x 1024, K = 4  (default: MegaTrain Table 4's
+              "MegaTrain (full)" setting, batch size 96)
   4 14b_x48   Qwen2.5-14B shape x 48 layers, batch 64 x 1024, K = 4
   5 7b_32k    7B shape x 28 layers, batch 1 x 32768, MLP in 4096-token chunks, K = 4
 
@@ -74,6 +75,39 @@ def load_peaks():
         d = json.load(open(p))
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def _flat_items(d, prefix=""):
+    for k, v in (d.items() if isinstance(d, dict) else []):
+        key = f"{prefix}.{k}" if prefix else str(k)
+        if isinstance(v, dict):
+            yield from _flat_items(v, key)
+        else:
+            yield key, v
+
+
+def sustained_peak_clock_mhz(peaks) -> tuple[float, str]:
+    """SM clock at which the sustained bf16 peak was taken: from the peaks file when it
+    records one, else the clock the profiling notes of this pool give for it (about 1.3 GHz
+    under the 1000 W power cap)."""
+    for k, v in _flat_items(peaks):
+        kl = k.lower()
+        if "sustain" in kl and ("mhz" in kl or "clock" in kl) and isinstance(v, (int, float)) and v > 100:
+            return float(v), k
+    return 1300.0, "assumed (sustained loop under the power cap)"
+
+
+def pick_peak(peaks, src, sm_mhz):
+    """The bf16 denominator for kernels timed inside a step: the sustained peak, unless the
+    run's median SM clock is above the clock the sustained peak was taken at (the GPU was
+    not held at that clock), in which case the burst peak."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = float(peaks.get("bf16_tflops_sustained", burst))
+    clk, clk_src = sustained_peak_clock_mhz(peaks)
+    use_burst = sm_mhz is not None and sm_mhz > 1.05 * clk
+    return {"burst": burst, "sustained": sust, "chosen": burst if use_burst else sust,
+            "which": "bf16_tflops (burst)" if use_burst else "bf16_tflops_sustained",
+            "source": src, "sustained_clock_mhz": clk, "sustained_clock_source": clk_src}
 
 
 def gemm_source_hash() -> str:
@@ -215,12 +249,13 @@ def measure_link(torch, nbytes=1 << 30):
 
 
 # ---------------------------------------------------------------- CPU oracle sample
-def oracle_sample(cfg, budget_s=12.0):
-    """Times the float64 oracle (forward + backward of one layer of this
-    workload's shape) on a bounded token sample; returns (TFLOPS, desc, threads)."""
+def oracle_sample(cfg, budget_s=12.0, max_tokens=1024):
+    """Times the float64 oracle (forward + backward of one layer of this workload's
+    shape) on one sequence of up to ``max_tokens`` tokens; returns (TFLOPS, description,
+    threads, seconds per rep, tokens)."""
     from oracle import OracleCfg, layer_bwd, layer_fwd
     sh = cfg["shape"]
-    T = min(cfg["T"], 256)
+    T = min(cfg["T"], max_tokens)
     B = 1
     ocfg = OracleCfg(**sh)
     shapes = synth.layer_tensor_shapes(**sh)
@@ -239,7 +274,20 @@ def oracle_sample(cfg, budget_s=12.0):
             break
     threads = os.environ.get("OPENBLAS_NUM_THREADS") or os.environ.get("OMP_NUM_THREADS") or str(os.cpu_count())
     desc = f"1 layer of the workload's shape, forward+backward, batch {B} x {T} tokens, {reps} reps in {el:.1f} s"
-    return flops * reps / el / 1e12, desc, int(threads), el / reps
+    return flops * reps / el / 1e12, desc, int(threads), el / reps, T
+
+
+def oracle_step_extrapolated(cfg, p_layer, sec, T_s):
+    """The oracle's time for one whole step of the workload (forward + backward of every
+    layer on all B x T tokens, no recompute), extrapolated from one layer on T_s tokens:
+    the sample's time is split in proportion to its projection FLOPs (6 P T_s) and
+    attention FLOPs (12 H T_s^2); the first part scales with the tokens B T, the second
+    with B T^2, and both with the layer count."""
+    H = cfg["shape"]["hidden"]
+    lin, att = 6.0 * p_layer * T_s, 12.0 * H * T_s ** 2
+    t_lin, t_att = sec * lin / (lin + att), sec * att / (lin + att)
+    B, T = cfg["B"], cfg["T"]
+    return cfg["L"] * (t_lin * B * T / T_s + t_att * B * (T / T_s) ** 2)
 
 
 def run_reference(args, cfg, rank, world):
@@ -248,7 +296,7 @@ def run_reference(args, cfg, rank, world):
         return
     vals = []
     for i in range(args.warmup + args.steps):
-        tf, desc, threads, sec = oracle_sample(cfg, budget_s=max(1.0, 20.0 / max(1, args.steps + args.warmup)))
+        tf, desc, threads, sec, _ = oracle_sample(cfg, budget_s=max(1.0, 20.0 / max(1, args.steps + args.warmup)))
         if i >= args.warmup:
             vals.append(tf)
     v = statistics.median(vals)
@@ -410,26 +458,44 @@ def run_ours(args, cfg, rank, world, local_rank):
     st = L_.mt_engine_stats(eng)  # the last timed step
     for _ in range(1):
         host_step()
-    ms_e2e = timed(host_step, max(1, args.steps // 2))
+    ms_e2e = timed(host_step, max(2, args.steps // 5))
     st_e2e = L_.mt_engine_stats(eng)
     assert L_.mt_device_error(clear=True) == 0, "a kernel's bounded wait ran out"
+    # one more step, outside every timed region, on an engine over the same memory with the event
+    # timeline on: per-phase device times and the transfer time the compute stream waited for
+    L_.mt_engine_destroy(eng)
+    topts = L_.mt_engine_opts.from_buffer_copy(opts)
+    topts.trace = 1
+    eng = L_.mt_engine_create(lcfg, nL, B, T, topts, ws, nbytes, *streams)
+    dev_step()
+    torch.cuda.synchronize()
+    st_tr = L_.mt_engine_stats(eng)
+    if args.trace and rank == 0:
+        with open(args.trace, "w") as f:
+            json.dump({"workload": cfg["name"], "intervals": L_.mt_engine_trace(eng)}, f, indent=0)
     link = measure_link(torch) if rank == 0 else None
 
     mflops = model_flops(cfg, p_layer, VOCAB if args.full_model else 0)
     value = job_throughput(mflops, world, ms) / 1e12
     e2e = job_throughput(mflops, world, ms_e2e) / 1e12
     peaks, src = load_peaks()
-    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    pk = pick_peak(peaks, src, clk.get("sm_mhz"))
+    peak_tf = pk["chosen"]
     gemm_tf = st.gemm_flops / (st.gemm_ms / 1e3) / 1e12 if st.gemm_ms > 0 else None
     line = None
     if rank == 0:
         bw = link
-        t_comp = st.exec_flops / (peak_tf * 1e12)
         t_h2d = st.h2d_bytes / (bw["h2d_gbs"] * 1e9)
         t_d2h = st.d2h_bytes / (bw["d2h_gbs"] * 1e9)
         t_bi = (st.h2d_bytes + st.d2h_bytes) / (bw["bidir_gbs"] * 1e9)
-        t_roof = max(t_comp, t_h2d, t_d2h, t_bi)
-        cpu_tf, cpu_desc, cpu_threads, _ = oracle_sample(cfg, budget_s=12.0)
+
+        def t_roof_at(peak):
+            return max(st.exec_flops / (peak * 1e12), t_h2d, t_d2h, t_bi)
+
+        t_comp = st.exec_flops / (peak_tf * 1e12)
+        t_roof = t_roof_at(peak_tf)
+        cpu_tf, cpu_desc, cpu_threads, cpu_sec, cpu_T = oracle_sample(cfg, budget_s=12.0)
+        tr = st_tr.trace
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -450,31 +516,34 @@ def run_ours(args, cfg, rank, world, local_rank):
             "roofline": {"bound": "tensor", "kernel": "gemm2_kernel (tcgen05, 2-SM)", "achieved": gemm_tf,
                          "peak": peak_tf, "unit": "TFLOP/s", "frac": (gemm_tf / peak_tf) if gemm_tf else None,
                          "traffic": gemm_traffic(cfg["name"]), "traffic_unit": "bytes per launch",
-                         "peak_source": f"{src} bf16_tflops_sustained",
+                         "peak_source": f"{src} {pk['which']}",
+                         "frac_of_burst": (gemm_tf / pk["burst"]) if gemm_tf else None,
+                         "frac_of_sustained": (gemm_tf / pk["sustained"]) if gemm_tf else None,
+                         "peak_rule": ("sustained peak unless the run's median SM clock exceeds the clock it was "
+                                       f"taken at ({pk['sustained_clock_mhz']:.0f} MHz, "
+                                       f"{pk['sustained_clock_source']})"),
                          "gemm_launches_per_step": int(st.gemm_launches)},
             "step_roofline": {"t_roof_ms": t_roof * 1e3, "t_step_ms": ms, "frac": t_roof / (ms / 1e3),
+                              "frac_at_burst_peak": t_roof_at(pk["burst"]) / (ms / 1e3),
+                              "frac_at_sustained_peak": t_roof_at(pk["sustained"]) / (ms / 1e3),
                               "t_compute_ms": t_comp * 1e3, "t_h2d_ms": t_h2d * 1e3, "t_d2h_ms": t_d2h * 1e3,
                               "t_bidir_ms": t_bi * 1e3, "exec_tflop": st.exec_flops / 1e12,
                               "model_tflop": mflops / 1e12, "h2d_bytes": int(st.h2d_bytes),
                               "d2h_bytes": int(st.d2h_bytes), "link_gbs": bw,
                               "model_flops_frac": mflops / (ms / 1e3) / (peak_tf * 1e12)},
+            "timeline": {"source": "one traced step after the timed ones (CUDA events around every upload, layer "
+                                   "call and offload)",
+                         "step_ms": tr.span_ms, "fwd_ms": tr.fwd_ms, "refwd_ms": tr.refwd_ms, "bwd_ms": tr.bwd_ms,
+                         "h2d_ms": tr.h2d_ms, "d2h_ms": tr.d2h_ms, "exposed_h2d_ms": tr.exposed_h2d_ms,
+                         "exposed_d2h_ms": tr.exposed_d2h_ms, "idle_other_ms": tr.idle_other_ms},
             "cpu_baseline": {"value": cpu_tf, "unit": UNIT, "cores": cpu_threads, "kind": "oracle",
-                             "sample": cpu_desc},
+                             "sample": cpu_desc,
+                             "step_s_extrapolated": oracle_step_extrapolated(cfg, p_layer, cpu_sec, cpu_T),
+                             "extrapolation": ("the oracle's forward+backward of every layer on all B x T tokens "
+                                               "(no recompute), scaled from the sample: projections linearly in "
+                                               "tokens, attention in B x T^2 (extrapolated, not measured)")},
             "device_workspace_gb": nbytes / 1e9,
         }
-    if args.trace:
-        # one more engine over the same memory, with the event timeline on: two steps, the last one's
-        # uploads, layer calls and offloads written to the trace file (outside every timed region)
-        L_.mt_engine_destroy(eng)
-        topts = L_.mt_engine_opts.from_buffer_copy(opts)
-        topts.trace = 1
-        eng = L_.mt_engine_create(lcfg, nL, B, T, topts, ws, nbytes, *streams)
-        for _ in range(2):
-            dev_step()
-        torch.cuda.synchronize()
-        if rank == 0:
-            with open(args.trace, "w") as f:
-                json.dump({"workload": cfg["name"], "intervals": L_.mt_engine_trace(eng)}, f, indent=0)
     L_.mt_engine_destroy(eng)
     if opt is not None:
         L_.mt_host_optimizer_destroy(opt)
@@ -491,7 +560,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
+    ap.add_argument("--config", type=int, default=3, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--full-model", action="store_true",
                     help="add the embedding and the final norm + LM head + loss (vocabulary 152064) to the step")

@@ -54,12 +54,23 @@ class mt_trace_rec(ctypes.Structure):
 TRACE_KINDS = ("h2d", "forward", "reforward", "backward", "d2h")
 
 
+class mt_trace_summary(ctypes.Structure):
+    _fields_ = [("span_ms", ctypes.c_double), ("h2d_ms", ctypes.c_double), ("d2h_ms", ctypes.c_double),
+                ("fwd_ms", ctypes.c_double), ("refwd_ms", ctypes.c_double), ("bwd_ms", ctypes.c_double),
+                ("exposed_h2d_ms", ctypes.c_double), ("exposed_d2h_ms", ctypes.c_double),
+                ("idle_other_ms", ctypes.c_double)]
+
+    def as_dict(self) -> dict:
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
 class mt_stats(ctypes.Structure):
-    _fields_ = [("step_ms", ctypes.c_double), ("h2d_ms", ctypes.c_double), ("d2h_ms", ctypes.c_double),
+    _fields_ = [("step_ms", ctypes.c_double),
                 ("h2d_bytes", c_u64), ("d2h_bytes", c_u64), ("layer_fwd_calls", c_u64), ("layer_bwd_calls", c_u64),
                 ("weight_loads", c_u64), ("exec_flops", ctypes.c_double), ("gemm_ms", ctypes.c_double),
                 ("gemm_flops", ctypes.c_double), ("gemm_launches", c_u64), ("device_bytes", c_u64),
-                ("sink_ms", ctypes.c_double), ("kernel_launches", c_u64)]
+                ("sink_ms", ctypes.c_double), ("kernel_launches", c_u64), ("traced", c_i32),
+                ("trace", mt_trace_summary)]
 
 
 class mt_adamw_cfg(ctypes.Structure):
@@ -110,6 +121,7 @@ _SIGS = {
     "mt_stream_step_hooked": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp, mt_head_hook, c_vp]),
     "mt_stream_step_host": (c_i32, [c_vp, c_vp, _P, _P, _P, _P, mt_grad_sink, c_vp]),
     "mt_engine_trace": (c_i32, [c_vp, ctypes.POINTER(mt_trace_rec), c_i32, ctypes.POINTER(c_i32)]),
+    "mt_trace_summarize": (c_i32, [ctypes.POINTER(mt_trace_rec), c_i32, ctypes.POINTER(mt_trace_summary)]),
     "mt_engine_stats": (c_i32, [c_vp, ctypes.POINTER(mt_stats)]),
     "mt_engine_reset": (c_i32, [c_vp]),
     "mt_engine_destroy": (None, [c_vp]),
@@ -354,6 +366,17 @@ def mt_engine_trace(engine, cap=4096) -> list:
     _check(load().mt_engine_trace(engine, recs, cap, ctypes.byref(n)))
     return [{"kind": TRACE_KINDS[r.kind], "layer": r.layer, "begin_ms": r.begin_ms, "end_ms": r.end_ms}
             for r in recs[:min(n.value, cap)]]
+
+
+def mt_trace_summarize(records) -> dict:
+    """Overlap summary of timeline records ({kind, layer, begin_ms, end_ms}, kinds named as
+    mt_engine_trace gives them): per-phase times and the exposed transfer time."""
+    arr = (mt_trace_rec * max(1, len(records)))()
+    for i, r in enumerate(records):
+        arr[i] = mt_trace_rec(TRACE_KINDS.index(r["kind"]), r["layer"], r["begin_ms"], r["end_ms"])
+    out = mt_trace_summary()
+    _check(load().mt_trace_summarize(arr, len(records), ctypes.byref(out)))
+    return out.as_dict()
 
 
 def mt_engine_reset(engine):

@@ -19,6 +19,7 @@
 // A second host thread polls d2h_done (bounded), hands each slab to the sink
 // in backward order and returns it to the pool. Every host wait is bounded by
 // the engine's timeout; nothing waits on the device.
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <cmath>
@@ -148,6 +149,74 @@ void mt_host_store_destroy(mt_host_store* s) {
 }
 
 }  // extern "C"
+
+// ======================================================================= timeline summary
+namespace {
+
+using Span = std::pair<double, double>;
+
+// Sorted, merged union of intervals.
+std::vector<Span> merged(std::vector<Span> v) {
+  std::sort(v.begin(), v.end());
+  std::vector<Span> out;
+  for (const Span& x : v) {
+    if (!out.empty() && x.first <= out.back().second)
+      out.back().second = std::max(out.back().second, x.second);
+    else
+      out.push_back(x);
+  }
+  return out;
+}
+
+// Whether instant t lies inside the merged union u.
+bool covers(const std::vector<Span>& u, double t) {
+  auto it = std::upper_bound(u.begin(), u.end(), Span(t, 1e300));
+  return it != u.begin() && t < std::prev(it)->second;
+}
+
+}  // namespace
+
+extern "C" mt_status mt_trace_summarize(const mt_trace_rec* recs, int32_t n, mt_trace_summary* out) {
+  if (!out || n < 0 || (n > 0 && !recs)) return fail(MT_ERR_INVALID_ARG, "trace_summarize: bad argument");
+  std::memset(out, 0, sizeof(*out));
+  std::vector<Span> comp, up, off;
+  std::vector<double> cuts = {0.0};
+  for (int i = 0; i < n; ++i) {
+    const mt_trace_rec& r = recs[i];
+    if (r.kind < 0 || r.kind > 4) return fail(MT_ERR_INVALID_ARG, "trace_summarize: unknown kind %d", r.kind);
+    if (!(r.end_ms >= r.begin_ms)) return fail(MT_ERR_INVALID_ARG, "trace_summarize: interval %d ends before it begins", i);
+    const double b = std::max(0.0, double(r.begin_ms)), e = std::max(0.0, double(r.end_ms));
+    const double d = e - b;
+    out->span_ms = std::max(out->span_ms, e);
+    switch (r.kind) {
+      case 0: out->h2d_ms += d; up.push_back({b, e}); break;
+      case 1: out->fwd_ms += d; comp.push_back({b, e}); break;
+      case 2: out->refwd_ms += d; comp.push_back({b, e}); break;
+      case 3: out->bwd_ms += d; comp.push_back({b, e}); break;
+      default: out->d2h_ms += d; off.push_back({b, e}); break;
+    }
+    cuts.push_back(b);
+    cuts.push_back(e);
+  }
+  comp = merged(comp);
+  up = merged(up);
+  off = merged(off);
+  std::sort(cuts.begin(), cuts.end());
+  // every elementary piece between consecutive boundaries is wholly inside or outside each union
+  for (size_t i = 0; i + 1 < cuts.size(); ++i) {
+    const double a = cuts[i], b = cuts[i + 1];
+    if (b <= a) continue;
+    const double mid = 0.5 * (a + b);
+    if (covers(comp, mid)) continue;
+    if (covers(up, mid))
+      out->exposed_h2d_ms += b - a;
+    else if (covers(off, mid))
+      out->exposed_d2h_ms += b - a;
+    else
+      out->idle_other_ms += b - a;
+  }
+  return MT_OK;
+}
 
 // ======================================================================= engine
 namespace {
@@ -361,6 +430,16 @@ void prepare_schedule(mt_engine* e) {
     e->load_of_use[i] = last_load[s];
     last_use[s] = i;
   }
+}
+
+// Interval k of the last traced step, in milliseconds from the step's origin.
+mt_status read_trace_rec(mt_engine* e, int k, mt_trace_rec* out) {
+  const auto& t = e->tr[k];
+  float b = 0.f, en = 0.f;
+  MT_CUDA(cudaEventElapsedTime(&b, e->tr_t0, e->tr_ev[t.eb]));
+  MT_CUDA(cudaEventElapsedTime(&en, e->tr_t0, e->tr_ev[t.ee]));
+  *out = {t.kind, t.layer, b, en};
+  return MT_OK;
 }
 
 mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const mt_bf16* dy_top, mt_bf16* y_top,
@@ -739,6 +818,16 @@ mt_status mt_stream_step_hooked(mt_engine* e, mt_host_store* store, const mt_bf1
   e->st.gemm_ms = 0;
   e->st.gemm_flops = 0;
   e->st.gemm_launches = 0;
+  e->st.traced = 0;
+  std::memset(&e->st.trace, 0, sizeof(e->st.trace));
+  if (s == MT_OK && e->opts.trace && e->tr_valid) {
+    std::vector<mt_trace_rec> recs(e->tr.size());
+    mt_status ts = MT_OK;
+    for (size_t k = 0; k < recs.size() && ts == MT_OK; ++k) ts = read_trace_rec(e, static_cast<int>(k), &recs[k]);
+    if (ts == MT_OK) ts = mt_trace_summarize(recs.data(), static_cast<int32_t>(recs.size()), &e->st.trace);
+    if (ts != MT_OK) return ts;
+    e->st.traced = 1;
+  }
   if (s == MT_OK && e->opts.time_gemms) {
     for (size_t k = 0; 2 * k + 1 < e->timer.n; ++k) {
       float ms = 0.f;
@@ -780,13 +869,7 @@ mt_status mt_engine_trace(mt_engine* e, mt_trace_rec* out, int32_t cap, int32_t*
   if (!e->opts.trace || !e->tr_valid)
     return fail(MT_ERR_INVALID_ARG, "engine_trace: the engine has no traced step (create it with trace = 1)");
   const int avail = static_cast<int>(e->tr.size());
-  for (int k = 0; k < avail && k < cap; ++k) {
-    const auto& t = e->tr[k];
-    float b = 0.f, en = 0.f;
-    MT_CUDA(cudaEventElapsedTime(&b, e->tr_t0, e->tr_ev[t.eb]));
-    MT_CUDA(cudaEventElapsedTime(&en, e->tr_t0, e->tr_ev[t.ee]));
-    out[k] = {t.kind, t.layer, b, en};
-  }
+  for (int k = 0; k < avail && k < cap; ++k) MT_TRY(read_trace_rec(e, k, &out[k]));
   *n = avail;
   return MT_OK;
 }

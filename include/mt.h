@@ -28,6 +28,9 @@
  * - Kernels that wait on barriers wait a bounded time; a wait that runs out
  *   sets a device error word (read with mt_device_error) and the kernel
  *   returns without finishing its output.
+ * - The library caches per-device state (kernel attributes, device addresses
+ *   of its own arrays) for the life of the process: no call may follow a
+ *   cudaDeviceReset of a device it has used.
  */
 #ifndef MT_H
 #define MT_H
@@ -300,9 +303,30 @@ typedef int32_t (*mt_grad_sink)(int32_t layer, const float* host_slab, uint64_t 
 
 typedef struct mt_engine mt_engine;
 
+/* What a traced step's timeline says about overlap (mt_trace_summarize).
+ * Times in milliseconds on the device clock. The compute stream is "idle" at
+ * an instant inside the step when none of its layer calls is running; the
+ * idle time is attributed to the weight uploads when one is in flight then,
+ * else to the gradient offloads when one is in flight, else to neither. */
+typedef struct mt_trace_summary {
+  double span_ms;          /* step origin (0) to the end of the last interval */
+  double h2d_ms;           /* sum of the weight-upload intervals (all pieces of a record) */
+  double d2h_ms;           /* sum of the gradient-offload intervals (first piece's start to last piece's end) */
+  double fwd_ms, refwd_ms, bwd_ms;  /* compute-stream time of forwards, segment re-forwards, recompute+backward */
+  double exposed_h2d_ms;   /* compute stream idle while a weight upload is in flight */
+  double exposed_d2h_ms;   /* compute stream idle while a gradient offload but no upload is in flight
+                              (this includes the drain after the last backward) */
+  double idle_other_ms;    /* compute stream idle with no copy in flight (host enqueue, a loss-head hook) */
+} mt_trace_summary;
+
+/* Host-only (no CUDA): summarizes n timeline records (mt_trace_rec, any
+ * order; kinds 0-4 as mt_engine_trace gives them). MT_ERR_INVALID_ARG on a
+ * NULL pointer, n < 0, an unknown kind or an interval that ends before it
+ * begins. */
+mt_status mt_trace_summarize(const mt_trace_rec* recs, int32_t n, mt_trace_summary* out);
+
 typedef struct mt_stats {
   double step_ms;             /* host wall time of the last step */
-  double h2d_ms, d2h_ms;      /* reserved, 0 (per-copy device times: mt_engine_trace) */
   uint64_t h2d_bytes, d2h_bytes;
   uint64_t layer_fwd_calls, layer_bwd_calls, weight_loads;
   double exec_flops;          /* FLOPs the kernels executed in the last step */
@@ -312,6 +336,8 @@ typedef struct mt_stats {
   uint64_t device_bytes;      /* device workspace bytes the engine uses */
   double sink_ms;             /* host time inside the sink */
   uint64_t kernel_launches;   /* kernels the library launched in the last step */
+  int32_t traced;             /* 1 when `trace` below describes the last step (engine created with trace = 1) */
+  mt_trace_summary trace;     /* per-phase device times and exposed transfer time of the last step */
 } mt_stats;
 
 /* Device workspace the engine needs (weight slots, gradient staging,
@@ -353,8 +379,8 @@ mt_status mt_stream_step_host(mt_engine* e, mt_host_store* store, const mt_bf16*
                               const mt_bf16* dy_top_host, mt_bf16* y_top_host, mt_bf16* dx0_host,
                               mt_grad_sink sink, void* user);
 
-/* Counters of the engine's last step (mt_stats above; h2d_ms and d2h_ms stay 0: the copies are
- * timed by the trace below). MT_ERR_INVALID_ARG on NULL. */
+/* Counters of the engine's last step (mt_stats above; its `trace` part is filled when
+ * the engine was created with trace = 1). MT_ERR_INVALID_ARG on NULL. */
 mt_status mt_engine_stats(const mt_engine* e, mt_stats* out);
 /* The timeline of the engine's last completed step, in issue order (engine
  * created with trace = 1; call after mt_stream_step returned MT_OK). Writes

@@ -19,6 +19,27 @@ pytestmark = pytest.mark.gpu
 TINY = dict(hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=688)
 
 
+QWEN7B = dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944)
+
+_RECORDS = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _free_records():
+    yield
+    _RECORDS.clear()  # the 7B layers' float64 copies are 1.9 GB each
+
+
+def _records(shape, n_layers, seed):
+    """(bf16 record bits, float64 weights) of each layer, generated once per shape and seed."""
+    key = (tuple(sorted(shape.items())), seed)
+    have = _RECORDS.setdefault(key, [])
+    cfg = L.make_cfg(**shape)
+    while len(have) < n_layers:
+        have.append(H.layer_record(cfg, seed, len(have), gain_std=0.1))
+    return have[:n_layers]
+
+
 class Stack:
     """Host store + engine for one configuration (seeded synthetic weights)."""
 
@@ -29,16 +50,15 @@ class Stack:
         self.store = L.mt_host_store_create(self.cfg, n_layers, True)
         off = L.mt_layer_param_offsets(self.cfg)
         self.rec_elems = off.record_elems
-        self.w64 = []
-        for l in range(n_layers):
-            rec, w64 = H.layer_record(self.cfg, seed, l, gain_std=0.1)
-            self.w64.append(w64)
+        recs = _records(shape, n_layers, seed)
+        self.w64 = [w64 for _, w64 in recs]
+        for l, (rec, _) in enumerate(recs):
             master = np.ctypeslib.as_array((ctypes.c_float * rec.size).from_address(L.mt_host_store_master(self.store, l)))
             master[:] = synth.bf16_bits_to_f32(rec)  # bf16-representable values: RNE keeps them
         L.mt_host_store_refresh_bf16(self.store, 0)
-        for l in range(n_layers):
+        for l, (rec, _) in enumerate(recs):
             bf = np.ctypeslib.as_array((ctypes.c_uint16 * self.rec_elems).from_address(L.mt_host_store_bf16(self.store, l)))
-            assert np.array_equal(bf, H.layer_record(self.cfg, seed, l, gain_std=0.1)[0])
+            assert np.array_equal(bf, rec)
         self.opts = L.make_opts(**opts)
         nbytes = L.mt_engine_workspace_bytes(self.cfg, n_layers, B, T, self.opts)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
@@ -69,6 +89,27 @@ class Stack:
     def close(self):
         L.mt_engine_destroy(self.eng)
         L.mt_host_store_destroy(self.store)
+        del self.ws
+
+
+def _check_against_oracle(s, y, dx, grads):
+    """Y, dX, the residual branch and every layer's gradient record against the oracle's stack."""
+    ocfg = H.oracle_cfg(s.cfg)
+    x64 = H.bits_to_f64(s.x)
+    y_ref, dx_ref, g_ref = O.stack_fwd_bwd(ocfg, s.w64, x64, H.bits_to_f64(s.dy))
+    errs = {"Y": H.rel(H.host_f64(y), y_ref), "dX": H.rel(H.host_f64(dx), dx_ref)}
+    bad = {k: v for k, v in errs.items() if not v < H.TOL}
+    br = H.rel(H.host_f64(y) - x64, y_ref - x64)
+    if not br < H.branch_tol(x64, y_ref):
+        bad["Y-X"] = br
+    assert sorted(grads) == list(range(s.L))
+    for l in range(s.L):
+        got = H.grads_from_record(s.cfg, grads[l])
+        for k, v in g_ref[l].items():
+            e = H.rel(got[k], v)
+            if not e < H.TOL:
+                bad[f"layer{l}.d{k}"] = e
+    assert not bad, bad
 
 
 def _as_bits(t):
@@ -81,17 +122,7 @@ def test_streamed_step_matches_oracle(n_layers, K):
     s = Stack(TINY, n_layers, 2, 128, ckpt_interval=K)
     try:
         y, dx, grads = s.step()
-        ocfg = H.oracle_cfg(s.cfg)
-        y_ref, dx_ref, g_ref = O.stack_fwd_bwd(ocfg, s.w64, H.bits_to_f64(s.x), H.bits_to_f64(s.dy))
-        assert H.rel(H.host_f64(y), y_ref) < H.TOL
-        x64 = H.bits_to_f64(s.x)
-        assert H.rel(H.host_f64(y) - x64, y_ref - x64) < H.branch_tol(x64, y_ref)
-        assert H.rel(H.host_f64(dx), dx_ref) < H.TOL
-        assert sorted(grads) == list(range(n_layers))
-        for l in range(n_layers):
-            got = H.grads_from_record(s.cfg, grads[l])
-            for k, v in g_ref[l].items():
-                assert H.rel(got[k], v) < H.TOL, (l, k)
+        _check_against_oracle(s, y, dx, grads)
         st = L.mt_engine_stats(s.eng)
         assert st.layer_bwd_calls == n_layers
         assert st.d2h_bytes == n_layers * s.rec_elems * 4
@@ -99,11 +130,23 @@ def test_streamed_step_matches_oracle(n_layers, K):
         s.close()
 
 
-def test_streamed_schedules_are_bit_exact_to_resident():
+def test_streamed_7b_shape_step_matches_oracle():
+    """Three Qwen2.5-7B-shaped layers on 1 x 1024 tokens with K = 2 (a re-forwarded
+    segment, a recomputed one and the top layer's reuse): the tcgen05 attention,
+    the 2-SM GEMMs at the layer's real widths and the engine's piecewise weight
+    upload and gradient offload at 7B record sizes, against the oracle per tensor."""
+    s = Stack(QWEN7B, 3, 1, 1024, ckpt_interval=2)
+    try:
+        y, dx, grads = s.step()
+        _check_against_oracle(s, y, dx, grads)
+    finally:
+        s.close()
+
+
+def _bit_exact_runs(shape, n_layers, B, T, K, variants):
     runs = {}
-    for name, opts in {"resident": dict(resident=1), "double": dict(), "single": dict(n_weight_slots=1),
-                       "pool1": dict(n_host_slabs=1, n_dev_grad_slabs=1), "nopool": dict(no_slab_pool=1)}.items():
-        s = Stack(TINY, 5, 2, 128, ckpt_interval=2, **opts)
+    for name, opts in variants.items():
+        s = Stack(shape, n_layers, B, T, ckpt_interval=K, **opts)
         try:
             y, dx, g = s.step()
             y2, dx2, g2 = s.step()  # a second step reuses every buffer
@@ -119,6 +162,25 @@ def test_streamed_schedules_are_bit_exact_to_resident():
         assert np.array_equal(dx, ref[1]), name
         for l in ref[2]:
             assert np.array_equal(g[l].view(np.uint32), ref[2][l].view(np.uint32)), (name, l)
+
+
+def test_7b_shape_streamed_schedules_are_bit_exact_to_resident():
+    """At the 7B layer shape: double-buffered streaming, a single weight slot and the
+    pool-less offload give the resident run's Y, dX and gradient records bit for bit."""
+    _bit_exact_runs(QWEN7B, 3, 1, 1024, 2, {"resident": dict(resident=1), "double": dict(),
+                                             "single": dict(n_weight_slots=1), "nopool": dict(no_slab_pool=1)})
+
+
+def test_7b_shape_b8_streamed_is_bit_exact_to_resident():
+    """8 x 1024 tokens: the weight-gradient GEMMs run the 256 x 512 tile (K = 8192)."""
+    _bit_exact_runs(QWEN7B, 3, 8, 1024, 2, {"resident": dict(resident=1), "double": dict()})
+
+
+def test_streamed_schedules_are_bit_exact_to_resident():
+    _bit_exact_runs(TINY, 5, 2, 128, 2, {"resident": dict(resident=1), "double": dict(),
+                                          "single": dict(n_weight_slots=1),
+                                          "pool1": dict(n_host_slabs=1, n_dev_grad_slabs=1),
+                                          "nopool": dict(no_slab_pool=1)})
 
 
 def test_host_buffer_step_equals_device_step():
@@ -337,6 +399,14 @@ def test_traced_step_gives_an_ordered_timeline():
         fwd = [r for r in tl if r["kind"] == "forward"]
         assert [r["layer"] for r in fwd] == list(range(5))
         assert all(a["end_ms"] <= b["begin_ms"] + 1e-3 for a, b in zip(fwd, fwd[1:]))  # one compute stream
+        # the stats carry the timeline's summary: per-phase device times and exposed transfer time
+        st = L.mt_engine_stats(s.eng)
+        assert st.traced == 1
+        tr = st.trace.as_dict()
+        assert tr == pytest.approx(L.mt_trace_summarize(tl))
+        busy = tr["fwd_ms"] + tr["refwd_ms"] + tr["bwd_ms"]
+        assert busy > 0 and tr["h2d_ms"] > 0 and tr["d2h_ms"] > 0
+        assert busy + tr["exposed_h2d_ms"] + tr["exposed_d2h_ms"] + tr["idle_other_ms"] == pytest.approx(tr["span_ms"])
         # tracing changes no result
         y1, dx1, g1 = s.step()
         assert np.array_equal(_as_bits(y0), _as_bits(y1)) and np.array_equal(_as_bits(dx0), _as_bits(dx1))

@@ -263,3 +263,54 @@ def test_attention_forward_and_backward(B, T, nq, nkv, d):
     L.mt_attention_bwd(qkv_d, ld, o, H.dev_bf16(do), nq * d, lse, dqkv2, B, T, nq, nkv, d, ws, ws.numel())
     torch.cuda.synchronize()
     assert torch.equal(dqkv.view(torch.int16), dqkv2.view(torch.int16))
+    # backward from the oracle's own o (rounded to bf16) and lse: independent of the forward kernel
+    _attention_bwd_from_oracle_forward(qkv_d, q, k, v, o_ref, lse_ref, do, B, T, nq, nkv, d)
+
+
+def _attention_bwd_from_oracle_forward(qkv_d, q, k, v, o_ref, lse_ref, do_bits, B, T, nq, nkv, d):
+    """The backward kernel fed the oracle forward's o (bf16) and lse (fp32), against the
+    oracle's backward on the same o and lse."""
+    import torch
+    ld = (nq + 2 * nkv) * d
+    o_bits = synth.f32_to_bf16_bits(o_ref.reshape(B, T, nq * d).astype(np.float32))
+    lse_f32 = np.ascontiguousarray(lse_ref, dtype=np.float32)
+    dqkv = torch.zeros(B, T, ld, dtype=torch.bfloat16, device="cuda")
+    ws = H.workspace(L.mt_attention_bwd_workspace_bytes(B, T, nq))
+    L.mt_attention_bwd(qkv_d, ld, H.dev_bf16(o_bits), H.dev_bf16(do_bits), nq * d, H.dev_f32(lse_f32), dqkv, B, T, nq,
+                       nkv, d, ws, ws.numel())
+    torch.cuda.synchronize()
+    _check_dev_error()
+    dq, dk, dv = O.attention_bwd(H.bits_to_f64(do_bits).reshape(B, T, nq, d), q, k, v,
+                                 H.bits_to_f64(o_bits).reshape(B, T, nq, d), lse_f32.astype(np.float64))
+    got = H.host_f64(dqkv)
+    errs = {"dq": H.rel(got[..., :nq * d], dq.reshape(B, T, -1)),
+            "dk": H.rel(got[..., nq * d:(nq + nkv) * d], dk.reshape(B, T, -1)),
+            "dv": H.rel(got[..., (nq + nkv) * d:], dv.reshape(B, T, -1))}
+    assert all(e < 2e-2 for e in errs.values()), errs
+
+
+@pytest.mark.parametrize("T", [8192, 16320])
+def test_long_context_attention_matches_oracle(T):
+    """Long sequences (the long-context workloads' regime): 64 and 128 key blocks per query
+    row, a group of 7 query heads per key/value head (the 7B ratio) and, at 16320 tokens, a
+    ragged last query block. Forward against the oracle; backward from the oracle's own
+    forward outputs against the oracle's backward."""
+    import torch
+    B, nq, nkv, d = 1, 7, 1, 128
+    ld = (nq + 2 * nkv) * d
+    qkv = _bits(12, T, B * T * ld, 1.5).reshape(B, T, ld)
+    do = _bits(13, T, B * T * nq * d).reshape(B, T, nq * d)
+    qkv_d = H.dev_bf16(qkv)
+    o = H.empty_bf16(B, T, nq * d)
+    lse = H.empty_f32(B, nq, T)
+    L.mt_attention_fwd(qkv_d, ld, o, nq * d, lse, B, T, nq, nkv, d)
+    torch.cuda.synchronize()
+    _check_dev_error()
+    q64 = H.bits_to_f64(qkv)
+    q = q64[..., :nq * d].reshape(B, T, nq, d)
+    k = q64[..., nq * d:(nq + nkv) * d].reshape(B, T, nkv, d)
+    v = q64[..., (nq + nkv) * d:].reshape(B, T, nkv, d)
+    o_ref, lse_ref = O.attention_fwd(q, k, v)
+    assert H.rel(H.host_f64(o), o_ref.reshape(B, T, nq * d)) < 1e-2
+    assert H.rel(H.host_f64(lse), lse_ref) < 1e-4
+    _attention_bwd_from_oracle_forward(qkv_d, q, k, v, o_ref, lse_ref, do, B, T, nq, nkv, d)

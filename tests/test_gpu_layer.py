@@ -25,8 +25,13 @@ CASES = {
     "mha": (dict(hidden=512, n_q_heads=4, n_kv_heads=4, head_dim=128, ffn=1376), 1, 200, 0),
     # the Qwen2.5-7B layer shape at reduced batch
     "qwen7b_b1_t128": (dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944), 1, 128, 0),
+    "qwen7b_b2_t128": (dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944), 2, 128, 0),
+    # one whole 1024-token sequence: eight 128-row query blocks per head, the persistent attention
+    # schedules, and every weight gradient summed over 1024 tokens
+    "qwen7b_b1_t1024": (dict(hidden=3584, n_q_heads=28, n_kv_heads=4, head_dim=128, ffn=18944), 1, 1024, 0),
     # the Qwen2.5-14B layer shape
     "qwen14b_b1_t64": (dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824), 1, 64, 0),
+    "qwen14b_b1_t1024": (dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824), 1, 1024, 0),
 }
 
 

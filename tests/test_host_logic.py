@@ -236,3 +236,55 @@ def test_gemm_traffic_is_tied_to_the_gemm_code_not_its_comments(tmp_path, monkey
     assert bench.gemm_source_hash() == h and bench.gemm_traffic("w") == 123.0
     g.write_text(g.read_text() + "static int changed_code = 1;\n")
     assert bench.gemm_source_hash() != h and bench.gemm_traffic("w") is None
+
+
+def test_trace_summary_attributes_idle_compute_to_the_copies_in_flight():
+    """A hand-made two-layer timeline: the compute stream waits 2 ms for the first upload,
+    runs, waits 1 ms for the second upload, runs the backward, then waits 1.5 ms for the
+    last gradient offload to drain; a 0.5 ms gap with nothing in flight counts as neither."""
+    recs = [
+        {"kind": "h2d", "layer": 0, "begin_ms": 0.0, "end_ms": 2.0},
+        {"kind": "h2d", "layer": 1, "begin_ms": 2.0, "end_ms": 5.0},
+        {"kind": "forward", "layer": 0, "begin_ms": 2.0, "end_ms": 4.0},
+        {"kind": "forward", "layer": 1, "begin_ms": 5.0, "end_ms": 6.0},
+        {"kind": "backward", "layer": 1, "begin_ms": 6.5, "end_ms": 9.0},
+        {"kind": "d2h", "layer": 1, "begin_ms": 8.0, "end_ms": 10.5},
+        {"kind": "reforward", "layer": 0, "begin_ms": 9.0, "end_ms": 9.25},
+        {"kind": "backward", "layer": 0, "begin_ms": 9.25, "end_ms": 10.0},
+        {"kind": "d2h", "layer": 0, "begin_ms": 10.0, "end_ms": 11.5},
+    ]
+    s = L.mt_trace_summarize(recs)
+    assert s["span_ms"] == pytest.approx(11.5)
+    assert s["h2d_ms"] == pytest.approx(5.0) and s["d2h_ms"] == pytest.approx(4.0)
+    assert s["fwd_ms"] == pytest.approx(3.0) and s["refwd_ms"] == pytest.approx(0.25)
+    assert s["bwd_ms"] == pytest.approx(3.25)
+    assert s["exposed_h2d_ms"] == pytest.approx(2.0 + 1.0)
+    assert s["exposed_d2h_ms"] == pytest.approx(1.5)
+    assert s["idle_other_ms"] == pytest.approx(0.5)
+    # every instant of the span is either compute or one of the three idle kinds
+    busy = s["fwd_ms"] + s["refwd_ms"] + s["bwd_ms"]
+    assert busy + s["exposed_h2d_ms"] + s["exposed_d2h_ms"] + s["idle_other_ms"] == pytest.approx(s["span_ms"])
+    assert L.mt_trace_summarize([])["span_ms"] == 0.0
+    with pytest.raises(L.MTError):
+        L.mt_trace_summarize([{"kind": "forward", "layer": 0, "begin_ms": 2.0, "end_ms": 1.0}])
+
+
+def test_bench_peak_choice_and_cpu_step_extrapolation():
+    """The bench takes the sustained bf16 peak unless the run's SM clock was above the clock
+    that peak was measured at, and extrapolates the oracle's step time from its sample
+    (exact when the sample is one layer of the workload itself)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    peaks = {"bf16_tflops": 1700.0, "bf16_tflops_sustained": 1400.0, "bf16_sustained_sm_mhz": 1350}
+    assert bench.pick_peak(peaks, "measured", 1300.0)["chosen"] == 1400.0
+    assert bench.pick_peak(peaks, "measured", 1950.0)["chosen"] == 1700.0
+    assert bench.pick_peak({"bf16_tflops": 1700.0}, "measured", None)["chosen"] == 1700.0
+    cfg = dict(shape=dict(hidden=3584), L=1, B=1, T=1024)
+    assert bench.oracle_step_extrapolated(cfg, 233_057_792, 2.0, 1024) == pytest.approx(2.0)
+    cfg28 = dict(shape=dict(hidden=3584), L=28, B=96, T=1024)
+    assert bench.oracle_step_extrapolated(cfg28, 233_057_792, 2.0, 1024) == pytest.approx(28 * 96 * 2.0)
+    # attention's share grows with T^2: doubling T more than doubles the step
+    long = dict(shape=dict(hidden=3584), L=1, B=1, T=2048)
+    assert bench.oracle_step_extrapolated(long, 233_057_792, 2.0, 1024) > 4.0

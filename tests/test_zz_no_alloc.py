@@ -65,12 +65,45 @@ def test_noalloc_rmsnorm_bwd_matches_workspace_entry_point_twice():
         assert torch.equal(dg, dg_ref)
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+def test_noalloc_at_its_exact_limit_matches_workspace_entry_point():
+    """ceil(rows / 64) * H = 2,097,152 exactly (16384 rows of 8192): the largest call the
+    fixed scratch takes, bit for bit equal to the workspace entry point."""
     import torch
-    rows, H = 64 * 600, 8192  # ceil(rows/64) * H = 4.9M > 2,097,152
+    rows, H = 16384, 8192
+
+    def bits(tid, n, std=1.0):
+        return synth.f32_to_bf16_bits(synth.normal_f32(78, 0, tid, n, std))
+    x, dy = _dev(bits(1, rows * H)), _dev(bits(2, rows * H))
+    g = _dev(synth.f32_to_bf16_bits((1.0 + synth.normal_f32(78, 0, 4, H, 0.2)).astype(np.float32)))
+    y = torch.empty_like(x)
+    rstd = torch.empty(rows, dtype=torch.float32, device="cuda")
+    L.mt_rmsnorm_fwd(x, g, y, rstd, rows, H, 1e-6)
+    del y
+    nws = L.mt_rmsnorm_bwd_workspace_bytes(rows, H)
+    assert nws == 8 << 20  # the scratch array's size
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    dx_ref = torch.empty_like(x)
+    dg_ref = torch.empty(H, dtype=torch.float32, device="cuda")
+    L.mt_rmsnorm_bwd(dy, x, g, rstd, None, dx_ref, dg_ref, rows, H, ws, nws)
+    dx = torch.full_like(x, float("nan"))
+    dg = torch.full((H,), float("nan"), dtype=torch.float32, device="cuda")
+    L.mt_rmsnorm_bwd_noalloc(dy, x, g, rstd, None, dx, dg, rows, H)
+    torch.cuda.synchronize()
+    assert L.mt_device_error(clear=True) == 0
+    assert torch.equal(dx.view(torch.int16), dx_ref.view(torch.int16))
+    assert torch.equal(dg, dg_ref)
+
+
+@pytest.mark.parametrize("rows,H", [(16385, 8192), (64 * 600, 8192)])  # one row past the limit, and far past it
+def test_noalloc_rejects_sizes_beyond_its_scratch_and_writes_nothing(rows, H):
+    import torch
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     r = torch.zeros(16, dtype=torch.float32, device="cuda")
+    dx = torch.full((16,), 3.0, dtype=torch.bfloat16, device="cuda")
+    dg = torch.full((16,), 5.0, dtype=torch.float32, device="cuda")
     with pytest.raises(L.MTError) as e:
-        L.mt_rmsnorm_bwd_noalloc(x, x, x, r, None, x, r, rows, H)
+        L.mt_rmsnorm_bwd_noalloc(x, x, x, r, None, dx, dg, rows, H)
     assert e.value.name == "MT_ERR_WORKSPACE"
     assert "scratch" in str(e.value)
+    torch.cuda.synchronize()
+    assert torch.all(dx == 3.0) and torch.all(dg == 5.0), "a rejected call wrote its outputs"

@@ -345,7 +345,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     abl = ABLATIONS[args.ablation]
     opts = L_.make_opts(ckpt_interval=abl.get("ckpt_interval", cfg["K"]), mlp_chunk=cfg["chunk"], time_gemms=1,
                         timeout_ms=120000, n_weight_slots=abl.get("n_weight_slots", 0),
-                        no_slab_pool=abl.get("no_slab_pool", 0))
+                        no_slab_pool=abl.get("no_slab_pool", 0), recompute_internals=int(args.recompute_internals))
     store = L_.mt_host_store_create(lcfg, nL, True)
     fill_store(L_, store, lcfg, nL)
     nbytes = L_.mt_engine_workspace_bytes(lcfg, nL, B, T, opts)
@@ -555,6 +555,99 @@ def run_ours(args, cfg, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- sweeps (MegaTrain Tables 5, 6, 7)
+def width_shape(scale: float) -> dict:
+    """The 7B layer widened by `scale` (MegaTrain Table 6 gives hidden and FFN sizes): head_dim 128
+    and the 7:1 query-to-key/value head ratio of the 7B shape are kept (the pages give no heads)."""
+    hidden = int(round(3584 * scale))
+    nq = hidden // 128
+    return dict(hidden=hidden, n_q_heads=nq, n_kv_heads=max(1, nq // 7), head_dim=128, ffn=int(round(18944 * scale)))
+
+
+SWEEPS = {
+    # Table 5: 7B width, depth 28 .. 180 layers
+    "depth": [dict(shape=QWEN7B, L=L, B=32, T=1024, K=4, chunk=0, label=f"7b_x{L}") for L in (28, 42, 56, 84, 132, 180)],
+    # Table 6: width 1.0x .. 3.5x at a fixed depth (12 layers: a 3.5x stack of 28 layers would need 160 GB of
+    # pinned bf16 weights, beyond the host memory of the GPU box next to the gradient slabs)
+    "width": [dict(shape=width_shape(w), L=12, B=32, T=1024, K=4, chunk=0, label=f"width{w}x_x12")
+              for w in (1.0, 1.5, 2.0, 2.5, 3.0, 3.5)],
+    # Table 7's longest rows: one sequence, MLP in 4096-token chunks (512K with the one-workspace schedule, whose
+    # per-layer internals of 21 GB would not fit K = 4 times next to the checkpoints)
+    "context": [dict(shape=QWEN7B, L=28, B=1, T=T, K=4, chunk=4096, label=f"7b_x28_b1x{T}",
+                     recompute_internals=int(T > 262144)) for T in (131072, 262144, 524288)],
+}
+
+
+def run_sweep(args, local_rank):
+    """Throughput of the streamed step across MegaTrain's depth, width and context studies. The host
+    store keeps only the bf16 streaming copy (no fp32 master: the sink does not update weights), filled
+    with one seeded block of 2^20 N(0, 0.02) values repeated over every record (the values do not change
+    the work); one JSON line per point, with the device memory the engine uses."""
+    import torch
+    from host_offloaded_layer_b200 import _lib as L_
+    torch.cuda.set_device(local_rank)
+    L_.load()
+    points = SWEEPS[args.sweep]
+    if args.points:
+        points = [points[i] for i in map(int, args.points.split(","))]
+    block = synth.f32_to_bf16_bits(synth.normal_f32(1234, 0, 99, 1 << 20, synth.WEIGHT_STD))
+    for pt in points:
+        sh, nL, B, T = pt["shape"], pt["L"], pt["B"], pt["T"]
+        lcfg = L_.make_cfg(**sh)
+        off = L_.mt_layer_param_offsets(lcfg)
+        p_layer = L_.mt_layer_param_count(lcfg)
+        opts = L_.make_opts(ckpt_interval=pt["K"], mlp_chunk=pt["chunk"], timeout_ms=600000,
+                            recompute_internals=pt.get("recompute_internals", 0))
+        store = L_.mt_host_store_create(lcfg, nL, False)
+        rec = np.resize(block, off.record_elems)
+        g1, g2 = int(off.g1), int(off.g2)
+        rec[g1:g1 + sh["hidden"]] = 0x3F80  # gains 1.0
+        rec[g2:g2 + sh["hidden"]] = 0x3F80
+        for l in range(nL):
+            dst = np.ctypeslib.as_array((ctypes.c_uint16 * off.record_elems).from_address(L_.mt_host_store_bf16(store, l)))
+            dst[:] = rec
+        nbytes = L_.mt_engine_workspace_bytes(lcfg, nL, B, T, opts)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        streams = [torch.cuda.Stream() for _ in range(3)]
+        eng = L_.mt_engine_create(lcfg, nL, B, T, opts, ws, nbytes, *streams)
+        H = sh["hidden"]
+        x_d = torch.from_numpy(synth.activations_bf16_bits(1234, synth.X0_ID, B, T, H).view(np.int16)).cuda()
+        dy_d = torch.from_numpy(synth.activations_bf16_bits(1234, synth.DY_ID, B, T, H).view(np.int16)).cuda()
+        y_d, dx_d = torch.empty_like(x_d), torch.empty_like(x_d)
+        step = lambda: L_.mt_stream_step(eng, store, x_d, dy_d, y_d, dx_d)  # noqa: E731
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(local_rank)
+        clocks.start()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(streams[0])
+        for _ in range(args.steps):
+            step()
+        ev1.record(streams[0])
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        ms = ev0.elapsed_time(ev1) / args.steps
+        st = L_.mt_engine_stats(eng)
+        assert L_.mt_device_error(clear=True) == 0, "a kernel's bounded wait ran out"
+        mflops = metrics.model_flops(nL * p_layer, nL, H, B, T)
+        rec_b = int(off.record_elems)
+        persistent = (max(2, pt["K"]) * rec_b * 2 + 2 * rec_b * 4) / 1e9  # weight slots + gradient staging
+        print(json.dumps({
+            "sweep": args.sweep, "point": pt["label"], "layers": nL, "shape": sh, "batch": B, "seq_len": T,
+            "ckpt_interval": pt["K"], "mlp_chunk": pt["chunk"],
+            "recompute_internals": pt.get("recompute_internals", 0),
+            "params_b": nL * p_layer / 1e9, "tflops": mflops / (ms / 1e3) / 1e12, "tokens_per_s": B * T / (ms / 1e3),
+            "step_s": ms / 1e3, "steps": args.steps, "warmup": args.warmup,
+            "exec_tflop_per_step": st.exec_flops / 1e12,
+            "device_workspace_gb": nbytes / 1e9, "device_weights_and_grad_staging_gb": persistent,
+            "host_pinned_gb": (nL * rec_b * 2 + 3 * rec_b * 4) / 1e9, "clocks": clk}), flush=True)
+        L_.mt_engine_destroy(eng)
+        L_.mt_host_store_destroy(store)
+        del ws, x_d, dy_d, y_d, dx_d
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -570,9 +663,18 @@ def main():
                     help="what receives each layer's gradient record (adamw: the CPU optimizer step)")
     ap.add_argument("--ablation", default="none", choices=sorted(ABLATIONS),
                     help="engine variant of MegaTrain Table 4 (default: the full system)")
+    ap.add_argument("--recompute-internals", action="store_true",
+                    help="every backward recomputes its layer's internals (one layer workspace, less memory)")
+    ap.add_argument("--sweep", default="", choices=["", *SWEEPS],
+                    help="instead of the benchmark line: one JSON line per point of the depth (Table 5), width "
+                         "(Table 6) or long-context (Table 7) study")
+    ap.add_argument("--points", default="", help="with --sweep: comma-separated indices of the points to run")
     args = ap.parse_args()
     rank, world, local_rank = dist_env()
     cfg = CONFIGS[args.config]
+    if args.sweep:
+        run_sweep(args, local_rank)
+        return
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
     else:

@@ -44,7 +44,7 @@ class mt_param_offsets(ctypes.Structure):
 class mt_engine_opts(ctypes.Structure):
     _fields_ = [(n, c_i32) for n in ("ckpt_interval", "n_weight_slots", "n_host_slabs", "n_dev_grad_slabs",
                                      "mlp_chunk", "resident", "timeout_ms", "fail_h2d_at", "time_gemms",
-                                     "no_slab_pool", "trace")]
+                                     "no_slab_pool", "trace", "recompute_internals")]
 
 
 class mt_trace_rec(ctypes.Structure):
@@ -315,9 +315,10 @@ def mt_host_store_destroy(store):
 
 
 def make_opts(ckpt_interval=4, n_weight_slots=0, n_host_slabs=0, n_dev_grad_slabs=0, mlp_chunk=0, resident=0,
-              timeout_ms=0, fail_h2d_at=0, time_gemms=0, no_slab_pool=0, trace=0) -> mt_engine_opts:
+              timeout_ms=0, fail_h2d_at=0, time_gemms=0, no_slab_pool=0, trace=0,
+              recompute_internals=0) -> mt_engine_opts:
     return mt_engine_opts(ckpt_interval, n_weight_slots, n_host_slabs, n_dev_grad_slabs, mlp_chunk, resident,
-                          timeout_ms, fail_h2d_at, time_gemms, no_slab_pool, trace)
+                          timeout_ms, fail_h2d_at, time_gemms, no_slab_pool, trace, recompute_internals)
 
 
 def mt_engine_workspace_bytes(cfg, n_layers, B, T, opts) -> int:

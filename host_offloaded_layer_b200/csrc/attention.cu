@@ -19,7 +19,8 @@
 namespace mt {
 
 mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o, int64_t ld_o, const float* lse,
-                             const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, cudaStream_t st);
+                             const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, const float* rope_tab,
+                             cudaStream_t st);
 
 namespace {
 
@@ -631,42 +632,48 @@ mt_status fwd_t(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t ld_o, float*
   return MT_OK;
 }
 
+// delta = rowsum(dO * O) per (row, head) into `delta` unless the caller already
+// formed it (have_delta), then dQ, dK, dV.
 template <int D>
 mt_status bwd_t(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, const mt_bf16* d_o, int64_t ld_o, const float* lse,
-                mt_bf16* dqkv, int B, int T, int nq, int nkv, float* delta, cudaStream_t st) {
-  using C = BwdCfg<D>;
-  static std::once_flag once;
-  static mt_status attr = MT_OK;
-  std::call_once(once, [] {
-    attr = set_smem(attn_bwd_dq_kernel<D>, C::SMEM);
-    if (attr == MT_OK) attr = set_smem(attn_bwd_dkv_kernel<D>, C::SMEM);
-  });
-  MT_TRY(attr);
-  const int64_t rows = static_cast<int64_t>(B) * T;
-  const int64_t n = rows * nq;
-  attn_delta_kernel<D><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, delta, rows, T, nq);
-  MT_TRY(launch_check("attn_delta_kernel"));
+                mt_bf16* dqkv, int B, int T, int nq, int nkv, float* delta, bool have_delta, const float* rope_tab,
+                cudaStream_t st) {
+  if (!have_delta) {
+    const int64_t rows = static_cast<int64_t>(B) * T;
+    const int64_t n = rows * nq;
+    attn_delta_kernel<D><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, delta, rows, T,
+        nq);
+    MT_TRY(launch_check("attn_delta_kernel"));
+  }
   if constexpr (D == 128) {
-    return attn_bwd_tc_launch(qkv, ld, d_o, ld_o, lse, delta, dqkv, B, T, nq, nkv, st);
+    return attn_bwd_tc_launch(qkv, ld, d_o, ld_o, lse, delta, dqkv, B, T, nq, nkv, rope_tab, st);
   } else {
-  const float scale = 1.0f / sqrtf(static_cast<float>(D));
-  const float scale_log2 = LOG2E * scale;
-  dim3 gq((T + C::BQ - 1) / C::BQ, nq, B);
-  attn_bwd_dq_kernel<D><<<gq, C::NT, C::SMEM, st>>>(reinterpret_cast<const __nv_bfloat16*>(qkv), ld,
-                                                    reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, lse, delta,
-                                                    reinterpret_cast<__nv_bfloat16*>(dqkv), T, nq, nkv, scale_log2,
-                                                    scale);
-  MT_TRY(launch_check("attn_bwd_dq_kernel"));
-  dim3 gk((T + C::BKV - 1) / C::BKV, nkv, B);
-  attn_bwd_dkv_kernel<D><<<gk, C::NT, C::SMEM, st>>>(reinterpret_cast<const __nv_bfloat16*>(qkv), ld,
-                                                     reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, lse, delta,
-                                                     reinterpret_cast<__nv_bfloat16*>(dqkv), T, nq, nkv, scale_log2,
-                                                     scale);
-  MT_TRY(launch_check("attn_bwd_dkv_kernel"));
-  // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)
-  add_exec_flops(14.0 * B * nq * D * (0.5 * double(T) * double(T)));
-  return MT_OK;
+    using C = BwdCfg<D>;
+    static std::once_flag once;
+    static mt_status attr = MT_OK;
+    std::call_once(once, [] {
+      attr = set_smem(attn_bwd_dq_kernel<D>, C::SMEM);
+      if (attr == MT_OK) attr = set_smem(attn_bwd_dkv_kernel<D>, C::SMEM);
+    });
+    MT_TRY(attr);
+    const float scale = 1.0f / sqrtf(static_cast<float>(D));
+    const float scale_log2 = LOG2E * scale;
+    dim3 gq((T + C::BQ - 1) / C::BQ, nq, B);
+    attn_bwd_dq_kernel<D><<<gq, C::NT, C::SMEM, st>>>(reinterpret_cast<const __nv_bfloat16*>(qkv), ld,
+                                                      reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, lse, delta,
+                                                      reinterpret_cast<__nv_bfloat16*>(dqkv), T, nq, nkv, scale_log2,
+                                                      scale);
+    MT_TRY(launch_check("attn_bwd_dq_kernel"));
+    dim3 gk((T + C::BKV - 1) / C::BKV, nkv, B);
+    attn_bwd_dkv_kernel<D><<<gk, C::NT, C::SMEM, st>>>(reinterpret_cast<const __nv_bfloat16*>(qkv), ld,
+                                                       reinterpret_cast<const __nv_bfloat16*>(d_o), ld_o, lse, delta,
+                                                       reinterpret_cast<__nv_bfloat16*>(dqkv), T, nq, nkv, scale_log2,
+                                                       scale);
+    MT_TRY(launch_check("attn_bwd_dkv_kernel"));
+    // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)
+    add_exec_flops(14.0 * B * nq * D * (0.5 * double(T) * double(T)));
+    return MT_OK;
   }
 }
 
@@ -693,8 +700,22 @@ mt_status attn_bwd_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* o, cons
                           cudaStream_t st) {
   if (B == 0 || T == 0) return MT_OK;
   float* delta = static_cast<float*>(ws);
-  if (d == 128) return bwd_t<128>(qkv, ld, o, d_o, ld_o, lse, dqkv, B, T, nq, nkv, delta, st);
-  if (d == 64) return bwd_t<64>(qkv, ld, o, d_o, ld_o, lse, dqkv, B, T, nq, nkv, delta, st);
+  if (d == 128) return bwd_t<128>(qkv, ld, o, d_o, ld_o, lse, dqkv, B, T, nq, nkv, delta, false, nullptr, st);
+  if (d == 64) return bwd_t<64>(qkv, ld, o, d_o, ld_o, lse, dqkv, B, T, nq, nkv, delta, false, nullptr, st);
+  return fail(MT_ERR_UNSUPPORTED, "attention supports head_dim 64 and 128, not %d", d);
+}
+
+// The attention backward of the layer: delta already formed (the dO GEMM's epilogue). For
+// head_dim 128, a non-NULL rope_tab makes dq and dk come out un-rotated; head_dim 64 takes
+// no table (its caller un-rotates with rope_launch).
+mt_status attn_bwd_delta_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o, int64_t ld_o, const float* lse,
+                                const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, int d,
+                                const float* rope_tab, cudaStream_t st) {
+  if (B == 0 || T == 0) return MT_OK;
+  float* dl = const_cast<float*>(delta);
+  if (d == 128) return bwd_t<128>(qkv, ld, nullptr, d_o, ld_o, lse, dqkv, B, T, nq, nkv, dl, true, rope_tab, st);
+  if (d == 64 && rope_tab) return fail(MT_ERR_UNSUPPORTED, "attention backward: un-rotation needs head_dim 128");
+  if (d == 64) return bwd_t<64>(qkv, ld, nullptr, d_o, ld_o, lse, dqkv, B, T, nq, nkv, dl, true, nullptr, st);
   return fail(MT_ERR_UNSUPPORTED, "attention supports head_dim 64 and 128, not %d", d);
 }
 

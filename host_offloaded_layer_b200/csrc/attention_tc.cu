@@ -520,7 +520,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
                            const __grid_constant__ CUtensorMap tm_do64, const float* __restrict__ lse,
                            const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int T,
-                           int nq, int nkv, float scale_log2, float scale, int32_t* err) {
+                           int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
+                           int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* lsd = reinterpret_cast<float*>(smem + KV_OFF_LD);  // [stage][lse2 | delta][64]
@@ -738,7 +739,36 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (ok && n_it > 0 && warp_wait(smem_u32(fin), 0, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) {
       fence_after();
       __nv_bfloat16* drow = dqkv + (static_cast<int64_t>(row0) + kv_row) * ld;
-      {
+      if (g == 0 && rope) {
+        // dK with the inverse rotation of its position: (a, b) -> (a cos + b sin, b cos - a sin)
+        // for the pair (i, i + 64), columns 32 cp + e and 32 cp + e + 64
+        __nv_bfloat16* out = drow + col_k;
+#pragma unroll
+        for (int cp = 0; cp < 2; ++cp) {
+          uint32_t ua[32], ub[32];
+          tmem_ld32(tmem + lane_base + KV_COL_DK + cp * 32, ua);
+          tmem_ld32(tmem + lane_base + KV_COL_DK + (cp + 2) * 32, ub);
+          if (kv_row < T) {
+            const float4* tab = reinterpret_cast<const float4*>(rope + static_cast<int64_t>(kv_row) * (D / 2) + cp * 32);
+            uint32_t pa[16], pb[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float4 cs = __ldg(tab + q);
+              const float a0 = __uint_as_float(ua[2 * q]) * scale, b0 = __uint_as_float(ub[2 * q]) * scale;
+              const float a1 = __uint_as_float(ua[2 * q + 1]) * scale, b1 = __uint_as_float(ub[2 * q + 1]) * scale;
+              pa[q] = pack_bf16(a0 * cs.x + b0 * cs.y, a1 * cs.z + b1 * cs.w);
+              pb[q] = pack_bf16(b0 * cs.x - a0 * cs.y, b1 * cs.z - a1 * cs.w);
+            }
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+              *reinterpret_cast<uint4*>(out + cp * 32 + qd * 8) =
+                  make_uint4(pa[4 * qd], pa[4 * qd + 1], pa[4 * qd + 2], pa[4 * qd + 3]);
+              *reinterpret_cast<uint4*>(out + (cp + 2) * 32 + qd * 8) =
+                  make_uint4(pb[4 * qd], pb[4 * qd + 1], pb[4 * qd + 2], pb[4 * qd + 3]);
+            }
+          }
+        }
+      } else {
         const int which = g;  // group 0 writes dK (scaled), group 1 dV
         const uint32_t col = which == 0 ? KV_COL_DK : KV_COL_DV;
         const float f = which == 0 ? scale : 1.f;
@@ -788,7 +818,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
                           const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
                           const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int B, int T,
-                          int nq, int nkv, float scale_log2, float scale, int32_t* err) {
+                          int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
+                          int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_SMEM_TILES);
@@ -1020,6 +1051,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       for (int ch = 0; ch < 2; ++ch) {  // group g writes dQ columns [64 g, 64 g + 64)
         uint32_t u[32];
         tmem_ld32(tmem + lane_base + DQ_COL_DQ + g * 64 + ch * 32, u);
+        if (rope) {
+          // the inverse rotation of the row's position pairs column i with i + 64, which the
+          // other group writes: read those partners too. Lower half (g = 0): a cos + b sin;
+          // upper half (g = 1): b cos - a sin, with a the lower and b the upper value.
+          uint32_t w[32];
+          tmem_ld32(tmem + lane_base + DQ_COL_DQ + (1 - g) * 64 + ch * 32, w);
+          if (q_row < T) {
+            const float4* tab = reinterpret_cast<const float4*>(rope + static_cast<int64_t>(q_row) * (D / 2) + ch * 32);
+            const float sg = g == 0 ? 1.f : -1.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float4 cs = __ldg(tab + q);
+              const float v0 = __uint_as_float(u[2 * q]), p0 = __uint_as_float(w[2 * q]);
+              const float v1 = __uint_as_float(u[2 * q + 1]), p1 = __uint_as_float(w[2 * q + 1]);
+              u[2 * q] = __float_as_uint(v0 * cs.x + sg * p0 * cs.y);
+              u[2 * q + 1] = __float_as_uint(v1 * cs.z + sg * p1 * cs.w);
+            }
+          }
+        }
         if (q_row < T) {
 #pragma unroll
           for (int qd = 0; qd < 4; ++qd) {
@@ -1048,8 +1098,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }  // namespace
 
 // dQ, dK, dV on the tensor cores (head_dim 128); delta = rowsum(dO * O) must be in `delta`.
+// With rope_tab (the (cos, sin) table of rope_table_launch) dq and dk come out with the
+// inverse rotation of their positions applied, i.e. as gradients of the unrotated q, k.
 mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o, int64_t ld_o, const float* lse,
-                             const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, cudaStream_t st) {
+                             const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, const float* rope_tab,
+                             cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -1074,12 +1127,13 @@ mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o,
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(dqkv);
   const int64_t dq_tiles = static_cast<int64_t>((T + 127) / 128) * nq * B;
   const int gq = static_cast<int>(std::min<int64_t>(dq_tiles, num_sms()));
+  const float2* rope = reinterpret_cast<const float2*>(rope_tab);
   attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, B, T, nq, nkv,
-                                                                scale_log2, scale, err);
+                                                                scale_log2, scale, rope, err);
   MT_TRY(launch_check("attn_bwd_dq_tc_kernel"));
   dim3 gk(nkv, B, (T + 127) / 128);
   attn_bwd_dkv_tc_kernel<<<gk, BWD_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, T, nq, nkv,
-                                                                 scale_log2, scale, err);
+                                                                 scale_log2, scale, rope, err);
   MT_TRY(launch_check("attn_bwd_dkv_tc_kernel"));
   // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)
   add_exec_flops(14.0 * B * nq * D * (0.5 * double(T) * double(T)));

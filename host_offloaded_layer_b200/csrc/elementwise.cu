@@ -180,6 +180,20 @@ __global__ void rope_kernel(__nv_bfloat16* x, int64_t ld, int64_t rows, int T, i
   }
 }
 
+// (cos, sin) of t * theta^(-2i/d) for every position t < T and pair i < d/2, formed
+// in fp64 like rope_kernel's and rounded to fp32: the table the RoPE epilogue of
+// the QKV projection reads.
+__global__ void rope_table_kernel(float2* tab, int64_t n, int half, int d, double theta) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= n) return;
+  const int64_t t = gid / half;
+  const int i = static_cast<int>(gid % half);
+  const double omega = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(d));
+  double sd, cd;
+  sincos(static_cast<double>(t) * omega, &sd, &cd);
+  tab[gid] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+}
+
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 
 __global__ void swiglu_fwd_kernel(const uint4* __restrict__ gu, uint4* __restrict__ m, int64_t rows, int F) {
@@ -291,6 +305,15 @@ mt_status rope_launch(mt_bf16* x, int64_t ld, int B, int T, int n_heads, int d, 
   rope_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(
       reinterpret_cast<__nv_bfloat16*>(x), ld, rows, T, n_heads, d, static_cast<double>(theta), inverse ? 1 : 0);
   return launch_check("rope_kernel");
+}
+
+mt_status rope_table_launch(float* tab, int T, int d, float theta, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(T) * (d / 2);
+  if (n == 0) return MT_OK;
+  const int threads = 256;
+  rope_table_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(
+      reinterpret_cast<float2*>(tab), n, d / 2, d, static_cast<double>(theta));
+  return launch_check("rope_table_kernel");
 }
 
 mt_status swiglu_fwd_launch(const mt_bf16* gu, mt_bf16* m, int64_t rows, int F, cudaStream_t st) {

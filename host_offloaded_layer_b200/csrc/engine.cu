@@ -44,9 +44,11 @@ mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt
                          int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep,
                          cudaEvent_t mlp_weights);
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
-                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd,
-                                 cudaEvent_t wd_done);
+                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws_int,
+                                 uint64_t int_bytes, void* ws_scr, uint64_t scr_bytes, void* stream,
+                                 cudaEvent_t mlp_done, bool reuse_fwd, cudaEvent_t wd_done);
+mt_status layer_ws_sizes(const mt_layer_cfg* cfg, int32_t B, int32_t T, int32_t mlp_chunk, uint64_t* internals,
+                         uint64_t* scratch);
 }  // namespace mt
 
 using namespace mt;
@@ -262,8 +264,11 @@ struct mt_engine {
   std::vector<float*> dgrad;
   std::vector<mt_bf16*> ckpt, seg;
   mt_bf16 *act[2] = {nullptr, nullptr}, *gbuf[2] = {nullptr, nullptr}, *io[4] = {nullptr, nullptr, nullptr, nullptr};
-  void* lws = nullptr;
-  uint64_t lws_bytes = 0, dev_bytes = 0;
+  // layer workspaces: internals sets (one per position in a segment, or one when every
+  // backward recomputes its layer's internals) and one scratch set for the backward
+  std::vector<void*> lws_int;
+  void* lws_scr = nullptr;
+  uint64_t int_bytes = 0, scr_bytes = 0, dev_bytes = 0;
   // host slab pool
   std::vector<float*> slab;
   std::mutex mu;
@@ -304,12 +309,20 @@ mt_bf16* x_loc(mt_engine* e, int j, const mt_bf16* x0, mt_bf16* ytop) {
   return e->act[j % 2];
 }
 
+// Layer-internals sets the engine carves: one per position in a segment, or one
+// when every backward recomputes its layer's internals.
+int internal_sets(const mt_engine_opts& o, int L) {
+  return o.recompute_internals ? 1 : std::min(o.ckpt_interval, L);
+}
+
 mt_status validate_opts(const mt_engine_opts* in, int L, mt_engine_opts* o) {
   if (!in) return fail(MT_ERR_INVALID_ARG, "opts is NULL");
   *o = *in;
   if (o->ckpt_interval < 1) return fail(MT_ERR_INVALID_ARG, "ckpt_interval must be >= 1");
   if (o->no_slab_pool < 0) return fail(MT_ERR_INVALID_ARG, "no_slab_pool must be 0 or 1");
   if (o->trace < 0 || o->trace > 1) return fail(MT_ERR_INVALID_ARG, "trace must be 0 or 1");
+  if (o->recompute_internals < 0 || o->recompute_internals > 1)
+    return fail(MT_ERR_INVALID_ARG, "recompute_internals must be 0 or 1");
   if (o->n_weight_slots < 0 || o->n_host_slabs < 0 || o->n_dev_grad_slabs < 0 || o->mlp_chunk < 0 ||
       o->timeout_ms < 0 || o->fail_h2d_at < 0)
     return fail(MT_ERR_INVALID_ARG, "engine options must be >= 0");
@@ -560,24 +573,38 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
       }
       if (status != MT_OK) break;
     }
-    // the backward of a layer that directly follows its own forward (the top layer) finds
-    // the forward's internals still in the layer workspace and skips their recompute
-    const bool fwd_then_bwd = i + 1 < n && u.kind == 0 && e->uses[i + 1].kind == 2 && e->uses[i + 1].layer == l;
-    const bool bwd_after_fwd = i > 0 && u.kind == 2 && e->uses[i - 1].kind == 0 && e->uses[i - 1].layer == l;
+    // Which forwards leave their internals for their backward, and so which backwards skip the
+    // recompute. Keeping (the default): every forward of the last segment and every segment
+    // re-forward keeps them in the internals set of its position in the segment; only the top
+    // layer of each earlier segment, which its re-forward does not reach, recomputes. With
+    // recompute_internals there is one set, and only the top layer, whose backward directly
+    // follows its forward, reuses it.
+    const int a_last = (e->S - 1) * e->K;
+    const int b_seg = std::min(e->L, a + e->K);
+    const bool keep_all = !e->opts.recompute_internals;
+    const int pos = keep_all ? l - a : 0;
+    bool keep = false, reuse = false;
+    if (keep_all) {
+      keep = u.kind == 1 || (u.kind == 0 && l >= a_last);
+      reuse = u.kind == 2 && (l >= a_last || l < b_seg - 1);
+    } else {
+      keep = i + 1 < n && u.kind == 0 && e->uses[i + 1].kind == 2 && e->uses[i + 1].layer == l;
+      reuse = i > 0 && u.kind == 2 && e->uses[i - 1].kind == 0 && e->uses[i - 1].layer == l;
+    }
+    void* lws = e->lws_int[pos];
     const int tk = tr_begin(u.kind + 1, l, e->cs);
     if (u.kind == 0) {
       // inside the last segment the forward keeps its activations in the segment buffers
-      const int a_last = (e->S - 1) * e->K;
       const mt_bf16* xin = (l > a_last) ? e->seg[l - a_last - 1] : x_loc(e, l, x0, y_top);
       mt_bf16* xout = (l + 1 < e->L && l + 1 > a_last) ? e->seg[l - a_last] : x_loc(e, l + 1, x0, y_top);
-      status = layer_fwd_keep(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes, e->cs,
-                              fwd_then_bwd, mlp_weights);
+      status = layer_fwd_keep(&e->cfg, w, xin, xout, e->B, e->T, e->opts.mlp_chunk, lws, e->int_bytes, e->cs, keep,
+                              mlp_weights);
       e->st.layer_fwd_calls++;
       tr_end(tk, e->cs);
     } else if (u.kind == 1) {
       const mt_bf16* xin = (l == a) ? x_loc(e, a, x0, y_top) : e->seg[l - a - 1];
-      status = layer_fwd_keep(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, e->lws, e->lws_bytes,
-                              e->cs, false, mlp_weights);
+      status = layer_fwd_keep(&e->cfg, w, xin, e->seg[l - a], e->B, e->T, e->opts.mlp_chunk, lws, e->int_bytes, e->cs,
+                              keep, mlp_weights);
       e->st.layer_fwd_calls++;
       tr_end(tk, e->cs);
     } else {
@@ -589,8 +616,9 @@ mt_status run_step(mt_engine* e, mt_host_store* store, const mt_bf16* x0, const 
         status = cuda_check(cudaStreamWaitEvent(e->cs, e->d2h_done[jb - e->NG], 0), "wait staging slab");
         if (status != MT_OK) break;
       }
-      status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, e->lws,
-                                      e->lws_bytes, e->cs, e->mlp_done[jb], bwd_after_fwd, e->wd_done[jb]);
+      status = layer_recompute_bwd_ev(&e->cfg, w, xin, dy, dx, e->dgrad[ns], e->B, e->T, e->opts.mlp_chunk, lws,
+                                      e->int_bytes, e->lws_scr, e->scr_bytes, e->cs, e->mlp_done[jb], reuse,
+                                      e->wd_done[jb]);
       e->st.layer_bwd_calls++;
       tr_end(tk, e->cs);
       if (status == MT_OK) status = cuda_check(cudaEventRecord(e->g_ready[jb], e->cs), "record g_ready");
@@ -687,9 +715,9 @@ uint64_t mt_engine_workspace_bytes(const mt_layer_cfg* cfg, int32_t n_layers, in
   mt_engine_opts o;
   if (make_geom(cfg, &G) != MT_OK || n_layers <= 0 || validate_opts(opts, n_layers, &o) != MT_OK) return 0;
   Bump bp = carve_engine(G, n_layers, B, T, o, nullptr, 0, nullptr);
-  const uint64_t lw = mt_layer_workspace_bytes(cfg, B, T, o.mlp_chunk);
-  if (lw == 0) return 0;
-  return bp.used + static_cast<uint64_t>(align_up(static_cast<int64_t>(lw), 256));
+  uint64_t wi = 0, wsc = 0;
+  if (layer_ws_sizes(cfg, B, T, o.mlp_chunk, &wi, &wsc) != MT_OK) return 0;
+  return bp.used + internal_sets(o, n_layers) * wi + wsc;
 }
 
 mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B, int32_t T,
@@ -728,8 +756,10 @@ mt_status mt_engine_create(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B,
   e->ps = as_stream(prefetch_stream);
   e->os = as_stream(offload_stream);
   Bump bp = carve_engine(G, n_layers, B, T, o, dev_ws, dev_ws_bytes, e);
-  e->lws = static_cast<char*>(dev_ws) + bp.used;
-  e->lws_bytes = dev_ws_bytes - bp.used;
+  MT_TRY(layer_ws_sizes(cfg, B, T, o.mlp_chunk, &e->int_bytes, &e->scr_bytes));
+  char* lw = static_cast<char*>(dev_ws) + bp.used;
+  for (int i = 0; i < internal_sets(o, n_layers); ++i, lw += e->int_bytes) e->lws_int.push_back(lw);
+  e->lws_scr = lw;
   e->dev_bytes = need;
   prepare_schedule(e);
   auto cleanup = [e](mt_status s) {

@@ -51,6 +51,11 @@ struct EpiArgs {
   int M, N, K;
   int c_f32, accumulate;
   int raster;
+  // raster 0: row-blocks per group. kalt = 1: a cluster's odd-numbered tiles walk K from
+  // the end down (so a wave starts on the K slices the previous wave read last, which
+  // are the ones still in L2); the fp32 summation order of a tile then depends on its
+  // place in the persistent walk, which is fixed for a given grid.
+  int group, kalt;
   // swiglu == 1, SwiGLU epilogue (2-SM kernel, both operands K-major): B holds
   // [Wg; Wu] (N = 2F rows); a pair tile covers 128 features j, C[m, j] =
   // silu(g) * u in bf16, and when gu is set g and u are also stored to gu[m, j]
@@ -61,12 +66,26 @@ struct EpiArgs {
   int swiglu, F;
   __nv_bfloat16* gu;
   int64_t ld_gu;
+  // rope_tab != NULL, RoPE epilogue (bf16 C, no residual): the first rope_cols
+  // columns are heads of rope_hd columns; after the bias, the pair (i, i + rope_hd/2)
+  // of each such head is rotated by the angle of position t = row % rope_T,
+  // (a, b) -> (a cos - b sin, b cos + a sin) with (cos, sin) = rope_tab[t * rope_hd/2 + i],
+  // and rounded to bf16 once.
+  const float2* rope_tab;
+  int rope_cols, rope_hd, rope_T;
+  // dot_with != NULL (bf16 C): per row r and head h of dot_hd columns, also
+  // dot_out[((r / dot_T) * dot_heads + h) * dot_T + r % dot_T] = sum_j C[r, j] * dot_with[r * ld_dot + j]
+  // over the head's columns, with C as stored (rounded to bf16), in fp32.
+  const __nv_bfloat16* dot_with;
+  int64_t ld_dot;
+  float* dot_out;
+  int dot_hd, dot_T, dot_heads;
 };
 
-// Output-tile order. raster 0: groups of 16 row-blocks, columns within a
+// Output-tile order. raster 0: groups of G row-blocks, columns within a
 // group; raster 1: row-major over all column blocks (the B operand stays in
 // L2); raster 2: column-major over all row blocks (the A operand stays in L2).
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int& mb, int& nb) {
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int G, int& mb, int& nb) {
   if (raster == 1) {
     mb = t / num_n;
     nb = t - mb * num_n;
@@ -77,7 +96,6 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
     mb = t - nb * num_m;
     return;
   }
-  constexpr int G = 16;
   const int group_tiles = G * num_n;
   const int g = t / group_tiles;
   const int first_m = g * G;
@@ -166,6 +184,82 @@ __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0
       }
     }
   }
+}
+
+// RoPE epilogue of one row: 32 columns of the first half of a head (clo, features
+// i0 .. i0 + 31 of the rotation) and their 32 partners of the second half (chi).
+__device__ __forceinline__ void store_rope_pair(const EpiArgs& ep, int row, int clo, int chi, int i0,
+                                                const uint32_t (&rl)[32], const uint32_t (&rh)[32]) {
+  float lo[32], hi[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    lo[j] = __uint_as_float(rl[j]);
+    hi[j] = __uint_as_float(rh[j]);
+  }
+  if (ep.bias) {
+    const uint4* bl = reinterpret_cast<const uint4*>(ep.bias + clo);
+    const uint4* bh = reinterpret_cast<const uint4*>(ep.bias + chi);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 ul = __ldg(bl + q), uh = __ldg(bh + q);
+      const __nv_bfloat16* hl = reinterpret_cast<const __nv_bfloat16*>(&ul);
+      const __nv_bfloat16* hh = reinterpret_cast<const __nv_bfloat16*>(&uh);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        lo[q * 8 + j] += bf2f(hl[j]);
+        hi[q * 8 + j] += bf2f(hh[j]);
+      }
+    }
+  }
+  const int t = row % ep.rope_T;
+  const float4* tab = reinterpret_cast<const float4*>(ep.rope_tab + static_cast<int64_t>(t) * (ep.rope_hd / 2) + i0);
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float4 cs = __ldg(tab + q);  // (cos, sin) of features i0 + 2q and i0 + 2q + 1
+    const float a0 = lo[2 * q], b0 = hi[2 * q], a1 = lo[2 * q + 1], b1 = hi[2 * q + 1];
+    lo[2 * q] = a0 * cs.x - b0 * cs.y;
+    hi[2 * q] = b0 * cs.x + a0 * cs.y;
+    lo[2 * q + 1] = a1 * cs.z - b1 * cs.w;
+    hi[2 * q + 1] = b1 * cs.z + a1 * cs.w;
+  }
+  __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 ul, uh;
+    __nv_bfloat162* pl = reinterpret_cast<__nv_bfloat162*>(&ul);
+    __nv_bfloat162* ph = reinterpret_cast<__nv_bfloat162*>(&uh);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      pl[j] = __floats2bfloat162_rn(lo[q * 8 + 2 * j], lo[q * 8 + 2 * j + 1]);
+      ph[j] = __floats2bfloat162_rn(hi[q * 8 + 2 * j], hi[q * 8 + 2 * j + 1]);
+    }
+    reinterpret_cast<uint4*>(crow + clo)[q] = ul;
+    reinterpret_cast<uint4*>(crow + chi)[q] = uh;
+  }
+}
+
+// bf16 store of one 32-column chunk (no bias or residual) that also returns
+// sum_j bf16(v_j) * dot_with[row, col0 + j] in fp32 (the dot epilogue).
+__device__ __forceinline__ float store_chunk_dot(const EpiArgs& ep, int row, int col0, const uint32_t (&r)[32]) {
+  uint4* cp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0);
+  const uint4* op = reinterpret_cast<const uint4*>(ep.dot_with + static_cast<int64_t>(row) * ep.ld_dot + col0);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 ov = op[q];
+    const __nv_bfloat162* ho = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      h[j] = __floats2bfloat162_rn(__uint_as_float(r[q * 8 + 2 * j]), __uint_as_float(r[q * 8 + 2 * j + 1]));
+      const float2 c = __bfloat1622float2(h[j]), o = __bfloat1622float2(ho[j]);
+      acc[q] = fmaf(c.x, o.x, acc[q]);
+      acc[q] = fmaf(c.y, o.y, acc[q]);
+    }
+    cp[q] = u;
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // SwiGLU backward of 32 features of one row from the fp32 dm accumulators:
@@ -417,9 +511,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     uint32_t it = 0;
     bool ok = true;
-    for (int t = cluster; t < num_tiles && ok; t += n_clusters) {
+    for (int t = cluster, tl = 0; t < num_tiles && ok; t += n_clusters, ++tl) {
       int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      tile_coords(t, num_m, num_n, ep.raster, ep.group, mb, nb);
+      const bool krev = ep.kalt && (tl & 1);
       const int m_own = mb * BM + static_cast<int>(rank) * 128;  // this CTA's A rows
       // this CTA's B rows of N-half h (SwiGLU: the gate rows in the even CTA, the up rows in the odd one)
       auto n_base = [&](int h, int rk) {
@@ -435,7 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
         }
         if (lane == 0) {
           const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
-          const int k0 = kb * BK;
+          const int k0 = (krev ? num_kb - 1 - kb : kb) * BK;
           const int atoms = min(KA, (ep.K - k0 + 63) / 64);  // atoms wholly past K are not loaded
           if (rank == 0) {
             uint32_t bytes = rows_bytes(A_MN, mb * BM, ep.M) + rows_bytes(A_MN, mb * BM + 128, ep.M);
@@ -481,6 +576,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
         if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
         fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
+        const bool krev = ep.kalt && (tl & 1);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -491,7 +587,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
           fence_after();
           if (lane == 0) {
             const uint32_t a_base = smem_u32(sA + s * A_STAGE), b_base = smem_u32(sB + s * B_STAGE);
-            const int ksteps = 4 * min(KA, (ep.K - kb * BK + 63) / 64);
+            const int ksteps = 4 * min(KA, (ep.K - (krev ? num_kb - 1 - kb : kb) * BK + 63) / 64);
             for (int kk = 0; kk < ksteps; ++kk) {
               // K-major: atom kk/4, then 16 elements (32 bytes) per step inside the swizzled row.
               // MN-major: 16 K-rows (two 8-row groups of 1 KiB) per step; MN atoms KA*8 KiB apart.
@@ -523,7 +619,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
       const int ab = NACC == 2 ? (tl & 1) : 0;
       const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
       int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      tile_coords(t, num_m, num_n, ep.raster, ep.group, mb, nb);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
@@ -537,6 +633,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
           tmem_ld32(tbase + static_cast<uint32_t>(c * 32), rg);
           tmem_ld32(tbase + static_cast<uint32_t>(128 + c * 32), ru);
           if (row < ep.M) store_swiglu(ep, row, f0, rg, ru);
+        }
+      } else if (ep.rope_tab) {
+        // a head holds hcn chunks of 32 columns; chunk c pairs with chunk c + hcn / 2
+        // (tiles start on head boundaries: 256 columns are whole heads of 64 or 128)
+        const int hcn = ep.rope_hd / 32, half = hcn / 2;
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = nb * BN + hc * 256 + c * 32;
+          if (col0 >= ep.N) break;
+          const int within = c % hcn;
+          if (col0 < ep.rope_cols) {
+            if (within >= half) continue;  // done with its partner
+            uint32_t rl[32], rh[32];
+            tmem_ld32(tbase + static_cast<uint32_t>(c * 32), rl);
+            tmem_ld32(tbase + static_cast<uint32_t>((c + half) * 32), rh);
+            if (row < ep.M) store_rope_pair(ep, row, col0, col0 + half * 32, within * 32, rl, rh);
+          } else {
+            uint32_t r[32];
+            tmem_ld32(tbase + static_cast<uint32_t>(c * 32), r);
+            if (row < ep.M) store_chunk(ep, row, col0, r);
+          }
+        }
+      } else if (ep.dot_with) {
+        const int hcn = ep.dot_hd / 32;
+        float acc = 0.f;
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = nb * BN + hc * 256 + c * 32;
+          if (col0 >= ep.N) break;
+          uint32_t r[32];
+          tmem_ld32(tbase + static_cast<uint32_t>(c * 32), r);
+          if (row < ep.M) {
+            acc += store_chunk_dot(ep, row, col0, r);
+            if (c % hcn == hcn - 1) {  // the head's last chunk
+              const int h = col0 / ep.dot_hd;
+              const int sq = row / ep.dot_T, t = row - sq * ep.dot_T;
+              ep.dot_out[(static_cast<int64_t>(sq) * ep.dot_heads + h) * ep.dot_T + t] = acc;
+              acc = 0.f;
+            }
+          }
         }
       } else {
         for (int c = 0; c < 8; ++c) {
@@ -598,6 +732,23 @@ mt_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return MT_OK;
 }
 
+// Wave shape of the grouped tile order (raster 0). All clusters walk K in step, so a
+// wave of `clusters` tiles reads each of its distinct A and B panels (256 rows, all of
+// K) about once from DRAM. With a short K the panels of a 16-row group stay in L2 for
+// the whole group (16 x 256 x K x 2 bytes within 32 MB). With a long K nothing
+// survives a wave but its last K slices: then a wave covers whole rows of tiles
+// (clusters / num_n of them), so consecutive waves read the same B panels, and every
+// other wave walks K backwards, starting where the previous one left L2.
+void pick_group(EpiArgs& e, int num_n, int clusters) {
+  e.group = 16;
+  e.kalt = 0;
+  if (e.raster != 0) return;
+  const int64_t panel = int64_t(c2::BM) * e.K * 2;
+  if (16 * panel <= (32ll << 20)) return;
+  e.kalt = 1;
+  e.group = num_n <= clusters ? std::max(1, clusters / num_n) : 8;
+}
+
 // Largest number of 2-CTA clusters of gemm2_kernel that fit on the device at once.
 template <bool A_MN, bool B_MN, int KA, int NH>
 int max_pair_clusters() {
@@ -635,7 +786,9 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
   const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN, KA, NH>());
   int32_t* err = device_error_word();
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
-  gemm2_kernel<A_MN, B_MN, KA, NH><<<2 * clusters, threads2(NH), c2::SMEM_BYTES, st>>>(ta, tb, ep, err);
+  EpiArgs e = ep;
+  pick_group(e, num_n, clusters);
+  gemm2_kernel<A_MN, B_MN, KA, NH><<<2 * clusters, threads2(NH), c2::SMEM_BYTES, st>>>(ta, tb, e, err);
   return launch_check("gemm2_kernel");
 }
 
@@ -711,10 +864,18 @@ EpiArgs plain_epilogue(int64_t M, int64_t N, int64_t K) {
   ep.c_f32 = 0;
   ep.accumulate = 0;
   ep.raster = 0;
+  ep.group = 16;
+  ep.kalt = 0;
   ep.swiglu = 0;
   ep.F = 0;
   ep.gu = nullptr;
   ep.ld_gu = 0;
+  ep.rope_tab = nullptr;
+  ep.rope_cols = ep.rope_hd = ep.rope_T = 0;
+  ep.dot_with = nullptr;
+  ep.ld_dot = 0;
+  ep.dot_out = nullptr;
+  ep.dot_hd = ep.dot_T = ep.dot_heads = 0;
   return ep;
 }
 
@@ -744,6 +905,39 @@ mt_status gemm_swiglu_bwd_launch(const mt_bf16* A, int64_t lda, bool a_mn, const
   return gemm_dispatch(A, lda, a_mn, B, ldb, b_mn, ep, st);
 }
 
+mt_status gemm_rope_launch(const mt_bf16* A, int64_t lda, const mt_bf16* B, int64_t ldb, mt_bf16* C, int64_t ldc,
+                           int64_t M, int64_t N, int64_t K, const mt_bf16* bias, const float* rope_tab, int rope_cols,
+                           int head_dim, int T, cudaStream_t st) {
+  if (N % head_dim || rope_cols % head_dim || rope_cols > N || (head_dim != 64 && head_dim != 128) || T <= 0)
+    return fail(MT_ERR_UNSUPPORTED, "RoPE epilogue: whole heads of 64 or 128 columns");
+  EpiArgs ep = plain_epilogue(M, N, K);
+  ep.C = C;
+  ep.ldc = ldc;
+  ep.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  ep.rope_tab = reinterpret_cast<const float2*>(rope_tab);
+  ep.rope_cols = rope_cols;
+  ep.rope_hd = head_dim;
+  ep.rope_T = T;
+  return gemm_dispatch(A, lda, false, B, ldb, false, ep, st);
+}
+
+mt_status gemm_dot_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
+                          mt_bf16* C, int64_t ldc, int64_t M, int64_t N, int64_t K, const mt_bf16* dot_with,
+                          int64_t ld_dot, float* dot_out, int head_dim, int T, cudaStream_t st) {
+  if (N % head_dim || (head_dim != 64 && head_dim != 128) || T <= 0 || M % T)
+    return fail(MT_ERR_UNSUPPORTED, "dot epilogue: whole heads of 64 or 128 and whole sequences");
+  EpiArgs ep = plain_epilogue(M, N, K);
+  ep.C = C;
+  ep.ldc = ldc;
+  ep.dot_with = reinterpret_cast<const __nv_bfloat16*>(dot_with);
+  ep.ld_dot = ld_dot;
+  ep.dot_out = dot_out;
+  ep.dot_hd = head_dim;
+  ep.dot_T = T;
+  ep.dot_heads = static_cast<int>(N / head_dim);
+  return gemm_dispatch(A, lda, a_mn, B, ldb, b_mn, ep, st);
+}
+
 mt_status tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
                      uint32_t box_inner, uint32_t box_outer) {
   return make_map(m, ptr, inner, outer, ld_elems, box_inner, box_outer);
@@ -755,17 +949,9 @@ mt_status gemm_swiglu_launch(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, 
   CUtensorMap ta, tb;
   MT_TRY(make_map(&ta, A, K, M, lda, 64, 128));
   MT_TRY(make_map(&tb, Wgu, K, 2 * F, ldw, 64, 128));
-  EpiArgs ep;
+  EpiArgs ep = plain_epilogue(M, 2 * F, K);
   ep.C = m;
-  ep.bias = nullptr;
-  ep.res = nullptr;
   ep.ldc = ldm;
-  ep.ldr = 0;
-  ep.M = static_cast<int>(M);
-  ep.N = static_cast<int>(2 * F);
-  ep.K = static_cast<int>(K);
-  ep.c_f32 = 0;
-  ep.accumulate = 0;
   ep.raster = pick_raster(M, 2 * F, K);
   ep.swiglu = 1;
   ep.F = static_cast<int>(F);

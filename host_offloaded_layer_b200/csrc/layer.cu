@@ -19,12 +19,14 @@
 namespace mt {
 
 mt_status layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
-                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
-                                 uint64_t ws_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd,
-                                 cudaEvent_t wd_done);
+                                 mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws_int,
+                                 uint64_t int_bytes, void* ws_scr, uint64_t scr_bytes, void* stream,
+                                 cudaEvent_t mlp_done, bool reuse_fwd, cudaEvent_t wd_done);
 mt_status layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
-                         int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream, bool keep,
+                         int32_t T, int32_t mlp_chunk, void* ws_int, uint64_t int_bytes, void* stream, bool keep,
                          cudaEvent_t mlp_weights);
+mt_status layer_ws_sizes(const mt_layer_cfg* cfg, int32_t B, int32_t T, int32_t mlp_chunk, uint64_t* internals,
+                         uint64_t* scratch);
 mt_status rmsnorm_fwd_launch(const mt_bf16*, const mt_bf16*, mt_bf16*, float*, int64_t, int, float, cudaStream_t);
 mt_status rmsnorm_bwd_launch(const mt_bf16*, const mt_bf16*, const mt_bf16*, const float*, const mt_bf16*, mt_bf16*,
                              float*, int64_t, int, void*, cudaStream_t);
@@ -37,6 +39,9 @@ mt_status attn_fwd_launch(const mt_bf16*, int64_t, mt_bf16*, int64_t, float*, in
 mt_status attn_bwd_launch(const mt_bf16*, int64_t, const mt_bf16*, const mt_bf16*, int64_t, const float*, mt_bf16*,
                           int, int, int, int, int, void*, cudaStream_t);
 uint64_t attn_bwd_ws_bytes(int B, int T, int nq);
+mt_status attn_bwd_delta_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o, int64_t ld_o, const float* lse,
+                                const float* delta, mt_bf16* dqkv, int B, int T, int nq, int nkv, int d,
+                                const float* rope_tab, cudaStream_t st);
 mt_status gemm_swiglu_launch(const mt_bf16* A, int64_t lda, const mt_bf16* Wgu, int64_t ldw, mt_bf16* m, int64_t ldm,
                              mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st);
 
@@ -45,11 +50,16 @@ namespace {
 struct LayerWs {
   mt_bf16 *h1, *qkv, *o, *x2, *h2, *gu, *m;
   float *rstd1, *rstd2, *lse;
+  float* rope;  // (cos, sin) of every position and rotation pair: [T][d/2] float pairs
   mt_bf16 *dh2, *dx2, *d_o, *dqkv;  // dm reuses m, dgu reuses gu, dh1 reuses dh2
   float* red;
 };
 
-Bump carve(const Geom& G, int B, int T, int64_t Mc, void* base, uint64_t cap, LayerWs* w) {
+// The layer's workspace in two parts. The internals are what a forward leaves for
+// its backward (h1, qkv after RoPE, o, x2, h2, the MLP chunk's g|u and m, the two
+// rstd vectors, lse and the RoPE table); the scratch holds the backward's own
+// buffers. The forward uses only the internals.
+Bump carve_internals(const Geom& G, int B, int T, int64_t Mc, void* base, uint64_t cap, LayerWs* w) {
   const int64_t M = static_cast<int64_t>(B) * T;
   Bump bp(base, cap);
   w->h1 = bp.take<mt_bf16>(M * G.H);
@@ -62,6 +72,13 @@ Bump carve(const Geom& G, int B, int T, int64_t Mc, void* base, uint64_t cap, La
   w->rstd1 = bp.take<float>(M);
   w->rstd2 = bp.take<float>(M);
   w->lse = bp.take<float>(static_cast<int64_t>(B) * G.nq * T);
+  w->rope = bp.take<float>(static_cast<int64_t>(T) * G.d);
+  return bp;
+}
+
+Bump carve_scratch(const Geom& G, int B, int T, void* base, uint64_t cap, LayerWs* w) {
+  const int64_t M = static_cast<int64_t>(B) * T;
+  Bump bp(base, cap);
   w->dh2 = bp.take<mt_bf16>(M * G.H);
   w->dx2 = bp.take<mt_bf16>(M * G.H);
   w->d_o = bp.take<mt_bf16>(M * G.Nq);
@@ -89,10 +106,10 @@ mt_status attention_half(const Geom& G, const mt_bf16* w, const mt_bf16* x, int 
   const int64_t M = static_cast<int64_t>(B) * T;
   const mt_param_offsets& O = G.off;
   MT_TRY(rmsnorm_fwd_launch(x, w + O.g1, ws.h1, ws.rstd1, M, static_cast<int>(G.H), G.eps, st));
-  MT_TRY(gemm_launch(ws.h1, G.H, false, w + O.wq, G.H, false, ws.qkv, G.Nqkv, false, false, M, G.Nqkv, G.H,
-                     G.bias ? w + O.bq : nullptr, nullptr, 0, st));
-  MT_TRY(rope_launch(ws.qkv, G.Nqkv, B, T, static_cast<int>(G.nq + G.nkv), static_cast<int>(G.d), G.theta, false,
-                     st));
+  // qkv = h1 Wqkv^T + bqkv with q and k rotated in the GEMM's epilogue
+  MT_TRY(rope_table_launch(ws.rope, T, static_cast<int>(G.d), G.theta, st));
+  MT_TRY(gemm_rope_launch(ws.h1, G.H, w + O.wq, G.H, ws.qkv, G.Nqkv, M, G.Nqkv, G.H, G.bias ? w + O.bq : nullptr,
+                          ws.rope, static_cast<int>((G.nq + G.nkv) * G.d), static_cast<int>(G.d), T, st));
   MT_TRY(attn_fwd_launch(ws.qkv, G.Nqkv, ws.o, G.Nq, ws.lse, B, T, static_cast<int>(G.nq), static_cast<int>(G.nkv),
                          static_cast<int>(G.d), st));
   MT_TRY(gemm_launch(ws.o, G.Nq, false, w + O.wo, G.Nq, false, ws.x2, G.H, false, false, M, G.H, G.Nq, nullptr, x, G.H,
@@ -119,26 +136,51 @@ using namespace mt;
 extern "C" {
 
 uint64_t mt_layer_workspace_bytes(const mt_layer_cfg* cfg, int32_t B, int32_t T, int32_t mlp_chunk) {
-  Geom G;
-  if (check_layer_args(cfg, &G, B, T, mlp_chunk) != MT_OK) return 0;
-  LayerWs w;
-  Bump bp = carve(G, B, T, chunk_rows(static_cast<int64_t>(B) * T, mlp_chunk), nullptr, 0, &w);
-  return bp.used;
+  uint64_t a = 0, b = 0;
+  if (layer_ws_sizes(cfg, B, T, mlp_chunk, &a, &b) != MT_OK) return 0;
+  return a + b;
+}
+
+// The one workspace of the public entry points: internals first, then scratch.
+static mt_status split_ws(const mt_layer_cfg* cfg, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
+                          uint64_t ws_bytes, void** scr, uint64_t* int_bytes, uint64_t* scr_bytes, const char* who) {
+  MT_TRY(layer_ws_sizes(cfg, B, T, mlp_chunk, int_bytes, scr_bytes));
+  if (ws_bytes < *int_bytes + *scr_bytes)
+    return fail(MT_ERR_WORKSPACE, "%s: workspace %llu < %llu bytes", who, (unsigned long long)ws_bytes,
+                (unsigned long long)(*int_bytes + *scr_bytes));
+  *scr = ws ? static_cast<char*>(ws) + *int_bytes : nullptr;
+  return MT_OK;
 }
 
 mt_status mt_layer_fwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, mt_bf16* y, int32_t B,
                        int32_t T, int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream) {
-  return layer_fwd_keep(cfg, w_dev, x, y, B, T, mlp_chunk, ws, ws_bytes, stream, false, nullptr);
+  void* scr = nullptr;
+  uint64_t ni = 0, ns = 0;
+  MT_TRY(split_ws(cfg, B, T, mlp_chunk, ws, ws_bytes, &scr, &ni, &ns, "layer_fwd"));
+  return layer_fwd_keep(cfg, w_dev, x, y, B, T, mlp_chunk, ws, ni, stream, false, nullptr);
 }
 
 mt_status mt_layer_recompute_bwd(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x, const mt_bf16* dy,
                                  mt_bf16* dx, float* dw_dev, int32_t B, int32_t T, int32_t mlp_chunk, void* ws,
                                  uint64_t ws_bytes, void* stream) {
-  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ws_bytes, stream, nullptr, false,
-                                nullptr);
+  void* scr = nullptr;
+  uint64_t ni = 0, ns = 0;
+  MT_TRY(split_ws(cfg, B, T, mlp_chunk, ws, ws_bytes, &scr, &ni, &ns, "layer_recompute_bwd"));
+  return layer_recompute_bwd_ev(cfg, w_dev, x, dy, dx, dw_dev, B, T, mlp_chunk, ws, ni, scr, ns, stream, nullptr,
+                                false, nullptr);
 }
 
 }  // extern "C"
+
+mt_status mt::layer_ws_sizes(const mt_layer_cfg* cfg, int32_t B, int32_t T, int32_t mlp_chunk, uint64_t* internals,
+                             uint64_t* scratch) {
+  Geom G;
+  MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
+  LayerWs w;
+  *internals = carve_internals(G, B, T, chunk_rows(static_cast<int64_t>(B) * T, mlp_chunk), nullptr, 0, &w).used;
+  *scratch = carve_scratch(G, B, T, nullptr, 0, &w).used;
+  return MT_OK;
+}
 
 // The layer forward. With `keep` the workspace is left holding everything the
 // layer's backward would recompute (h1, qkv after RoPE, o, lse, x2, h2, and
@@ -158,7 +200,7 @@ mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, cons
   const int64_t M = static_cast<int64_t>(B) * T;
   const int64_t Mc = chunk_rows(M, mlp_chunk);
   LayerWs w;
-  Bump bp = carve(G, B, T, Mc, ws, ws_bytes, &w);
+  Bump bp = carve_internals(G, B, T, Mc, ws, ws_bytes, &w);
   if (!bp.ok()) return fail(MT_ERR_WORKSPACE, "layer_fwd: workspace %llu < %llu bytes", (unsigned long long)ws_bytes,
                             (unsigned long long)bp.used);
   cudaStream_t st = as_stream(stream);
@@ -181,21 +223,26 @@ mt_status mt::layer_fwd_keep(const mt_layer_cfg* cfg, const mt_bf16* w_dev, cons
 // ones it would produce: every kernel is deterministic).
 mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_dev, const mt_bf16* x,
                                      const mt_bf16* dy, mt_bf16* dx, float* dw_dev, int32_t B, int32_t T,
-                                     int32_t mlp_chunk, void* ws, uint64_t ws_bytes, void* stream,
-                                     cudaEvent_t mlp_done, bool reuse_fwd, cudaEvent_t wd_done) {
+                                     int32_t mlp_chunk, void* ws_int, uint64_t int_bytes, void* ws_scr,
+                                     uint64_t scr_bytes, void* stream, cudaEvent_t mlp_done, bool reuse_fwd,
+                                     cudaEvent_t wd_done) {
   Geom G;
   MT_TRY(check_layer_args(cfg, &G, B, T, mlp_chunk));
-  if (!w_dev || !x || !dy || !dx || !dw_dev || !ws) return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: NULL pointer");
-  if (!aligned16(w_dev) || !aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(dw_dev) || !aligned16(ws))
+  if (!w_dev || !x || !dy || !dx || !dw_dev || !ws_int || !ws_scr)
+    return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: NULL pointer");
+  if (!aligned16(w_dev) || !aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(dw_dev) ||
+      !aligned16(ws_int) || !aligned16(ws_scr))
     return fail(MT_ERR_ALIGNMENT, "layer_recompute_bwd: pointers must be 16-byte aligned");
   if (dx == x) return fail(MT_ERR_INVALID_ARG, "layer_recompute_bwd: dx must not alias x");
   const int64_t M = static_cast<int64_t>(B) * T;
   const int64_t Mc = chunk_rows(M, mlp_chunk);
   LayerWs w;
-  Bump bp = carve(G, B, T, Mc, ws, ws_bytes, &w);
-  if (!bp.ok())
-    return fail(MT_ERR_WORKSPACE, "layer_recompute_bwd: workspace %llu < %llu bytes", (unsigned long long)ws_bytes,
-                (unsigned long long)bp.used);
+  Bump bi = carve_internals(G, B, T, Mc, ws_int, int_bytes, &w);
+  Bump bs = carve_scratch(G, B, T, ws_scr, scr_bytes, &w);
+  if (!bi.ok() || !bs.ok())
+    return fail(MT_ERR_WORKSPACE, "layer_recompute_bwd: workspace %llu + %llu < %llu + %llu bytes",
+                (unsigned long long)int_bytes, (unsigned long long)scr_bytes, (unsigned long long)bi.used,
+                (unsigned long long)bs.used);
   cudaStream_t st = as_stream(stream);
   const mt_param_offsets& O = G.off;
   const int H = static_cast<int>(G.H);
@@ -229,12 +276,18 @@ mt_status mt::layer_recompute_bwd_ev(const mt_layer_cfg* cfg, const mt_bf16* w_d
   // dWo = dx2^T o ; do = dx2 Wo
   MT_TRY(gemm_launch(w.dx2, G.H, true, w.o, G.Nq, true, dw_dev + O.wo, G.Nq, true, false, G.H, G.Nq, M, nullptr,
                      nullptr, 0, st));
-  MT_TRY(gemm_launch(w.dx2, G.H, false, w_dev + O.wo, G.Nq, true, w.d_o, G.Nq, false, false, M, G.Nq, G.H, nullptr,
-                     nullptr, 0, st));
-  // attention backward -> dq, dk (rotated), dv; then un-rotate dq, dk
-  MT_TRY(attn_bwd_launch(w.qkv, G.Nqkv, w.o, w.d_o, G.Nq, w.lse, w.dqkv, B, T, static_cast<int>(G.nq),
-                         static_cast<int>(G.nkv), static_cast<int>(G.d), w.red, st));
-  MT_TRY(rope_launch(w.dqkv, G.Nqkv, B, T, static_cast<int>(G.nq + G.nkv), static_cast<int>(G.d), G.theta, true, st));
+  // do = dx2 Wo, and in the same GEMM's epilogue delta = rowsum(do * o) per head (the attention
+  // backward's D term), into the partial-sum buffer that the column sums reuse only later
+  MT_TRY(gemm_dot_launch(w.dx2, G.H, false, w_dev + O.wo, G.Nq, true, w.d_o, G.Nq, M, G.Nq, G.H, w.o, G.Nq, w.red,
+                         static_cast<int>(G.d), T, st));
+  // attention backward -> dq, dk, dv, with dq and dk un-rotated (the adjoint of RoPE) in the
+  // tcgen05 kernels' epilogues for head_dim 128, by a separate pass for head_dim 64
+  const bool d128 = G.d == 128;
+  MT_TRY(attn_bwd_delta_launch(w.qkv, G.Nqkv, w.d_o, G.Nq, w.lse, w.red, w.dqkv, B, T, static_cast<int>(G.nq),
+                               static_cast<int>(G.nkv), static_cast<int>(G.d), d128 ? w.rope : nullptr, st));
+  if (!d128)
+    MT_TRY(rope_launch(w.dqkv, G.Nqkv, B, T, static_cast<int>(G.nq + G.nkv), static_cast<int>(G.d), G.theta, true,
+                       st));
   if (G.bias) MT_TRY(colsum_launch(w.dqkv, nullptr, nullptr, M, G.Nqkv, G.Nqkv, dw_dev + O.bq, w.red, st));
   // dWqkv = dqkv^T h1 ; dh1 = dqkv Wqkv (into the dh2 buffer)
   MT_TRY(gemm_launch(w.dqkv, G.Nqkv, true, w.h1, G.H, true, dw_dev + O.wq, G.H, true, false, G.Nqkv, G.H, M, nullptr,

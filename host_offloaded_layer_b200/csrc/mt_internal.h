@@ -93,6 +93,22 @@ mt_status gemm_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B
 mt_status gemm_swiglu_bwd_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
                                  mt_bf16* gu, int64_t ld_gu, int64_t M, int64_t F, int64_t K, cudaStream_t st);
 
+// C = A B^T (both K-major, bf16 C) with bias and rotate-half RoPE applied to the
+// fp32 accumulators of the first rope_cols columns (heads of head_dim) at
+// position row % T; rope_tab holds (cos, sin) pairs, [T][head_dim / 2] (rope_table_launch).
+mt_status gemm_rope_launch(const mt_bf16* A, int64_t lda, const mt_bf16* B, int64_t ldb, mt_bf16* C, int64_t ldc,
+                           int64_t M, int64_t N, int64_t K, const mt_bf16* bias, const float* rope_tab, int rope_cols,
+                           int head_dim, int T, cudaStream_t st);
+
+// C = A B^T (bf16 C) that also writes, per row and head of head_dim columns, the
+// dot product of the stored C with dot_with into dot_out[seq][head][t] (fp32).
+mt_status gemm_dot_launch(const mt_bf16* A, int64_t lda, bool a_mn, const mt_bf16* B, int64_t ldb, bool b_mn,
+                          mt_bf16* C, int64_t ldc, int64_t M, int64_t N, int64_t K, const mt_bf16* dot_with,
+                          int64_t ld_dot, float* dot_out, int head_dim, int T, cudaStream_t st);
+
+// (cos, sin) of angle t * theta^(-2i/d) for t < T, i < d/2 as fp32 pairs, formed in fp64.
+mt_status rope_table_launch(float* tab, int T, int d, float theta, cudaStream_t st);
+
 // GEMM launch observer (engine statistics): called around each GEMM launch.
 struct GemmTimer {
   virtual void before(cudaStream_t st) = 0;

@@ -284,6 +284,11 @@ typedef struct mt_engine_opts {
                               (the "w/o Gradient Slab Pool" ablation of MegaTrain Table 4) */
   int32_t trace;           /* 1: time every weight upload, layer call and gradient offload of a
                               step with CUDA events (read back with mt_engine_trace) */
+  int32_t recompute_internals; /* 0 (default): a segment's re-forward (and the last segment's forward)
+                              keeps each layer's internals in a workspace of its own, min(K, L) of
+                              them, and the layer's backward reuses them; only the top layer of each
+                              earlier segment recomputes its internals. 1: one layer workspace, and
+                              every backward but the top layer's recomputes (less device memory). */
 } mt_engine_opts;
 
 /* One interval of a traced step (MegaTrain Fig. 3's timeline: H2D, compute and
@@ -341,7 +346,8 @@ typedef struct mt_stats {
 } mt_stats;
 
 /* Device workspace the engine needs (weight slots, gradient staging,
- * checkpoints, segment activations, one layer workspace). */
+ * checkpoints, segment activations, the layer internals sets of
+ * recompute_internals and one backward scratch). */
 uint64_t mt_engine_workspace_bytes(const mt_layer_cfg* cfg, int32_t n_layers, int32_t B, int32_t T,
                                    const mt_engine_opts* opts);
 

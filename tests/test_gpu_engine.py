@@ -146,7 +146,7 @@ def test_streamed_7b_shape_step_matches_oracle():
 def _bit_exact_runs(shape, n_layers, B, T, K, variants):
     runs = {}
     for name, opts in variants.items():
-        s = Stack(shape, n_layers, B, T, ckpt_interval=K, **opts)
+        s = Stack(shape, n_layers, B, T, **{"ckpt_interval": K, **opts})
         try:
             y, dx, g = s.step()
             y2, dx2, g2 = s.step()  # a second step reuses every buffer
@@ -168,7 +168,8 @@ def test_7b_shape_streamed_schedules_are_bit_exact_to_resident():
     """At the 7B layer shape: double-buffered streaming, a single weight slot and the
     pool-less offload give the resident run's Y, dX and gradient records bit for bit."""
     _bit_exact_runs(QWEN7B, 3, 1, 1024, 2, {"resident": dict(resident=1), "double": dict(),
-                                             "single": dict(n_weight_slots=1), "nopool": dict(no_slab_pool=1)})
+                                             "single": dict(n_weight_slots=1), "nopool": dict(no_slab_pool=1),
+                                             "recompute": dict(recompute_internals=1)})
 
 
 def test_7b_shape_b8_streamed_is_bit_exact_to_resident():
@@ -177,10 +178,15 @@ def test_7b_shape_b8_streamed_is_bit_exact_to_resident():
 
 
 def test_streamed_schedules_are_bit_exact_to_resident():
+    # recompute_internals: every backward recomputes its layer's internals instead of reusing the
+    # segment re-forward's; the kernels are deterministic, so the results are the same bits
     _bit_exact_runs(TINY, 5, 2, 128, 2, {"resident": dict(resident=1), "double": dict(),
                                           "single": dict(n_weight_slots=1),
                                           "pool1": dict(n_host_slabs=1, n_dev_grad_slabs=1),
-                                          "nopool": dict(no_slab_pool=1)})
+                                          "nopool": dict(no_slab_pool=1),
+                                          "recompute": dict(recompute_internals=1),
+                                          "recompute_k3": dict(recompute_internals=1, ckpt_interval=3),
+                                          "k3": dict(ckpt_interval=3)})
 
 
 def test_host_buffer_step_equals_device_step():

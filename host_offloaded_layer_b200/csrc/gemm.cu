@@ -51,11 +51,6 @@ struct EpiArgs {
   int M, N, K;
   int c_f32, accumulate;
   int raster;
-  // raster 0: row-blocks per group. kalt = 1: a cluster's odd-numbered tiles walk K from
-  // the end down (so a wave starts on the K slices the previous wave read last, which
-  // are the ones still in L2); the fp32 summation order of a tile then depends on its
-  // place in the persistent walk, which is fixed for a given grid.
-  int group, kalt;
   // swiglu == 1, SwiGLU epilogue (2-SM kernel, both operands K-major): B holds
   // [Wg; Wu] (N = 2F rows); a pair tile covers 128 features j, C[m, j] =
   // silu(g) * u in bf16, and when gu is set g and u are also stored to gu[m, j]
@@ -82,10 +77,10 @@ struct EpiArgs {
   int dot_hd, dot_T, dot_heads;
 };
 
-// Output-tile order. raster 0: groups of G row-blocks, columns within a
+// Output-tile order. raster 0: groups of 16 row-blocks, columns within a
 // group; raster 1: row-major over all column blocks (the B operand stays in
 // L2); raster 2: column-major over all row blocks (the A operand stays in L2).
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int G, int& mb, int& nb) {
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int& mb, int& nb) {
   if (raster == 1) {
     mb = t / num_n;
     nb = t - mb * num_n;
@@ -96,6 +91,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
     mb = t - nb * num_m;
     return;
   }
+  constexpr int G = 16;
   const int group_tiles = G * num_n;
   const int g = t / group_tiles;
   const int first_m = g * G;
@@ -511,10 +507,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     uint32_t it = 0;
     bool ok = true;
-    for (int t = cluster, tl = 0; t < num_tiles && ok; t += n_clusters, ++tl) {
+    for (int t = cluster; t < num_tiles && ok; t += n_clusters) {
       int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, ep.group, mb, nb);
-      const bool krev = ep.kalt && (tl & 1);
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       const int m_own = mb * BM + static_cast<int>(rank) * 128;  // this CTA's A rows
       // this CTA's B rows of N-half h (SwiGLU: the gate rows in the even CTA, the up rows in the odd one)
       auto n_base = [&](int h, int rk) {
@@ -530,7 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
         }
         if (lane == 0) {
           const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
-          const int k0 = (krev ? num_kb - 1 - kb : kb) * BK;
+          const int k0 = kb * BK;
           const int atoms = min(KA, (ep.K - k0 + 63) / 64);  // atoms wholly past K are not loaded
           if (rank == 0) {
             uint32_t bytes = rows_bytes(A_MN, mb * BM, ep.M) + rows_bytes(A_MN, mb * BM + 128, ep.M);
@@ -576,7 +571,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
         if (!warp_wait(smem_u32(&tempty[ab]), aph ^ 1u, abort_flag, err, DEV_ERR_TIMEOUT_MMA)) break;
         fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
-        const bool krev = ep.kalt && (tl & 1);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -587,7 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
           fence_after();
           if (lane == 0) {
             const uint32_t a_base = smem_u32(sA + s * A_STAGE), b_base = smem_u32(sB + s * B_STAGE);
-            const int ksteps = 4 * min(KA, (ep.K - (krev ? num_kb - 1 - kb : kb) * BK + 63) / 64);
+            const int ksteps = 4 * min(KA, (ep.K - kb * BK + 63) / 64);
             for (int kk = 0; kk < ksteps; ++kk) {
               // K-major: atom kk/4, then 16 elements (32 bytes) per step inside the swizzled row.
               // MN-major: 16 K-rows (two 8-row groups of 1 KiB) per step; MN atoms KA*8 KiB apart.
@@ -619,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
       const int ab = NACC == 2 ? (tl & 1) : 0;
       const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
       int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, ep.group, mb, nb);
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
@@ -732,23 +726,6 @@ mt_status make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return MT_OK;
 }
 
-// Wave shape of the grouped tile order (raster 0). All clusters walk K in step, so a
-// wave of `clusters` tiles reads each of its distinct A and B panels (256 rows, all of
-// K) about once from DRAM. With a short K the panels of a 16-row group stay in L2 for
-// the whole group (16 x 256 x K x 2 bytes within 32 MB). With a long K nothing
-// survives a wave but its last K slices: then a wave covers whole rows of tiles
-// (clusters / num_n of them), so consecutive waves read the same B panels, and every
-// other wave walks K backwards, starting where the previous one left L2.
-void pick_group(EpiArgs& e, int num_n, int clusters) {
-  e.group = 16;
-  e.kalt = 0;
-  if (e.raster != 0) return;
-  const int64_t panel = int64_t(c2::BM) * e.K * 2;
-  if (16 * panel <= (32ll << 20)) return;
-  e.kalt = 1;
-  e.group = num_n <= clusters ? std::max(1, clusters / num_n) : 8;
-}
-
 // Largest number of 2-CTA clusters of gemm2_kernel that fit on the device at once.
 template <bool A_MN, bool B_MN, int KA, int NH>
 int max_pair_clusters() {
@@ -786,9 +763,7 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
   const int clusters = std::min(num_tiles, max_pair_clusters<A_MN, B_MN, KA, NH>());
   int32_t* err = device_error_word();
   if (!err) return fail(MT_ERR_CUDA, "device error word unavailable");
-  EpiArgs e = ep;
-  pick_group(e, num_n, clusters);
-  gemm2_kernel<A_MN, B_MN, KA, NH><<<2 * clusters, threads2(NH), c2::SMEM_BYTES, st>>>(ta, tb, e, err);
+  gemm2_kernel<A_MN, B_MN, KA, NH><<<2 * clusters, threads2(NH), c2::SMEM_BYTES, st>>>(ta, tb, ep, err);
   return launch_check("gemm2_kernel");
 }
 
@@ -864,8 +839,6 @@ EpiArgs plain_epilogue(int64_t M, int64_t N, int64_t K) {
   ep.c_f32 = 0;
   ep.accumulate = 0;
   ep.raster = 0;
-  ep.group = 16;
-  ep.kalt = 0;
   ep.swiglu = 0;
   ep.F = 0;
   ep.gu = nullptr;

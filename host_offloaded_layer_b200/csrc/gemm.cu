@@ -770,13 +770,17 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
 // Pair-tile width. The 256 x 512 tile (NH = 2) measured 4-7% faster on the
 // weight-gradient layout (both operands MN-major, K = tokens >= 16384, fp32 out),
 // where a tile's main loop is long enough to hide its unbuffered epilogue, and
-// 2-5% slower on the forward and input-gradient shapes of the layer (K = 3584):
-// it is used for the weight-gradient layout with K >= 8192. Every other launch
-// runs the 256 x 256 tile with three stages of 128-wide K (eight MMAs per
-// barrier round trip measured 7-16% faster than four on every layout).
+// 2-5% slower on the forward and input-gradient shapes of the layer with K = 3584.
+// On the long-K forward / input-gradient launches (the down projection, K = F,
+// and dh2 = dgu Wgu, K = 2F) it measured 10-13% faster at 98304 rows but 4%
+// slower at 8192 (fewer tiles than two waves of clusters). So: the weight-gradient
+// layout with K >= 8192, and any plain epilogue with K >= 8192 and M >= 65536.
+// Every other launch runs the 256 x 256 tile with three stages of 128-wide K
+// (eight MMAs per barrier round trip measured 7-16% faster than four).
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
-  const bool wide = A_MN && B_MN && ep.swiglu == 0 && ep.K >= 8192;
+  const bool plain = ep.swiglu == 0 && !ep.rope_tab && !ep.dot_with;
+  const bool wide = plain && ep.K >= 8192 && ((A_MN && B_MN) || ep.M >= 65536);
   if (wide) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
   return launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st);
 }

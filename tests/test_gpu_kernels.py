@@ -81,6 +81,27 @@ def test_gemm_is_deterministic_and_covers_many_waves():
     _check_dev_error()
 
 
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1)])
+def test_gemm_long_k_many_rows_wide_tile(a_mn, b_mn):
+    """At 65536 rows and more with K >= 8192 the forward and input-gradient layouts run the
+    256 x 512 pair tile (the down projection and dh2 of the 96 x 1024 workload): sampled rows
+    of a bf16 result with a residual against the float64 product, and a ragged last row block."""
+    import torch
+    M, N, K = 65600, 384, 8200
+    A = _bits(13, 1, M * K).reshape(M, K)
+    b_rows, b_cols = (K, N) if b_mn else (N, K)
+    B = _bits(13, 2, b_rows * b_cols, 0.05).reshape(b_rows, b_cols)
+    res = _bits(13, 3, M * N).reshape(M, N)
+    C = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    L.mt_gemm_bf16(H.dev_bf16(A), K, a_mn, H.dev_bf16(B), b_cols, b_mn, C, N, 0, 0, M, N, K, None, H.dev_bf16(res), N)
+    torch.cuda.synchronize()
+    _check_dev_error()
+    rows = np.concatenate([np.random.default_rng(3).choice(M - 64, 60, replace=False), np.arange(M - 4, M)])
+    b64 = H.bits_to_f64(B)
+    ref = H.bits_to_f64(A[rows]) @ (b64 if b_mn else b64.T) + H.bits_to_f64(res[rows])
+    assert H.rel(H.host_f64(C)[rows], ref) < 1e-2
+
+
 @pytest.mark.parametrize("M,F,K", [(256, 688, 256), (200, 1000, 136), (8192, 18944, 3584)])
 def test_gemm_with_swiglu_epilogue(M, F, K):
     import torch

@@ -1,6 +1,8 @@
 """Times one block kernel through the C ABI (CUDA events, warm-up first).
 
     python -m host_offloaded_layer_b200.kernel_bench gemm --M 16384 --N 4608 --K 3584 --layout kk
+    python -m host_offloaded_layer_b200.kernel_bench gemm_swiglu --M 8192 --F 18944 --K 3584
+    python -m host_offloaded_layer_b200.kernel_bench gemm_swiglu_bwd --M 8192 --F 18944 --K 3584
     python -m host_offloaded_layer_b200.kernel_bench attn_fwd --B 8 --T 1024 --nq 28 --nkv 4 --d 128
     python -m host_offloaded_layer_b200.kernel_bench attn_bwd --B 8 --T 1024 --nq 28 --nkv 4 --d 128
     python -m host_offloaded_layer_b200.kernel_bench rmsnorm --rows 8192 --H 3584
@@ -32,7 +34,8 @@ def main():
     from host_offloaded_layer_b200 import _lib as L
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemm", "attn_fwd", "attn_bwd", "rmsnorm", "swiglu", "layer"])
+    ap.add_argument("op", choices=["gemm", "gemm_swiglu", "gemm_swiglu_bwd", "attn_fwd", "attn_bwd", "rmsnorm", "swiglu",
+                                   "layer"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=4608)
     ap.add_argument("--K", type=int, default=3584)
@@ -64,6 +67,23 @@ def main():
                                     stream=st)
         work, unit = 2.0 * a.M * a.N * a.K, "TFLOP/s"
         shape = dict(M=a.M, N=a.N, K=a.K, layout=a.layout, f32=a.f32)
+    elif a.op == "gemm_swiglu":
+        # the gate/up projection with the SwiGLU epilogue (m, and g and u for the backward)
+        A = _dev(torch, a.M * a.K, 1)
+        W = _dev(torch, 2 * a.F * a.K, 2, 0.02)
+        m = torch.empty(a.M * a.F, dtype=torch.bfloat16, device="cuda")
+        gu = torch.empty(a.M * 2 * a.F, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: L.mt_gemm_swiglu_bf16(A, a.K, W, a.K, m, a.F, gu, 2 * a.F, a.M, a.F, a.K, st)  # noqa: E731
+        work, unit = 2.0 * a.M * 2 * a.F * a.K, "TFLOP/s"
+        shape = dict(M=a.M, F=a.F, K=a.K)
+    elif a.op == "gemm_swiglu_bwd":
+        # dm = dY Wd with the SwiGLU backward over [g|u] in place
+        dY = _dev(torch, a.M * a.K, 1)
+        Wd = _dev(torch, a.K * a.F, 2, 0.02)
+        gu = _dev(torch, a.M * 2 * a.F, 3)
+        fn = lambda: L.mt_gemm_swiglu_bwd_bf16(dY, a.K, Wd, a.F, gu, 2 * a.F, a.M, a.F, a.K, st)  # noqa: E731
+        work, unit = 2.0 * a.M * a.F * a.K, "TFLOP/s"
+        shape = dict(M=a.M, F=a.F, K=a.K)
     elif a.op in ("attn_fwd", "attn_bwd"):
         ld = (a.nq + 2 * a.nkv) * a.d
         qkv = _dev(torch, a.B * a.T * ld, 1)

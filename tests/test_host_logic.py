@@ -288,3 +288,31 @@ def test_bench_peak_choice_and_cpu_step_extrapolation():
     # attention's share grows with T^2: doubling T more than doubles the step
     long = dict(shape=dict(hidden=3584), L=1, B=1, T=2048)
     assert bench.oracle_step_extrapolated(long, 233_057_792, 2.0, 1024) > 4.0
+
+
+def test_sweep_points_fit_the_device_and_the_host():
+    """Every point of bench.py's depth / width / context sweeps (MegaTrain Tables 5-7) sizes an engine
+    workspace that fits a B200's 180 GB and a pinned bf16 store plus gradient slabs within 190 GB of host
+    memory; the depth sweep's device workspace grows only by the checkpoint stash (one [B, T, H] bf16
+    activation per K layers)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    ws = {}
+    for sweep, points in bench.SWEEPS.items():
+        for pt in points:
+            cfg = L.make_cfg(**pt["shape"])
+            opts = L.make_opts(ckpt_interval=pt["K"], mlp_chunk=pt["chunk"],
+                               recompute_internals=pt.get("recompute_internals", 0))
+            n = L.mt_engine_workspace_bytes(cfg, pt["L"], pt["B"], pt["T"], opts)
+            rec = L.mt_layer_param_offsets(cfg).record_elems
+            assert 0 < n < 180e9, (sweep, pt["label"], n)
+            assert pt["L"] * rec * 2 + 3 * rec * 4 < 190e9, (sweep, pt["label"])
+            ws[(sweep, pt["L"])] = n
+    depth = sorted((L_, n) for (s, L_), n in ws.items() if s == "depth")
+    act = 32 * 1024 * 3584 * 2
+    for (l0, n0), (l1, n1) in zip(depth, depth[1:]):
+        assert n1 - n0 == ((l1 + 3) // 4 - (l0 + 3) // 4) * act
+    w = bench.width_shape(3.5)
+    assert (w["hidden"], w["ffn"], w["n_q_heads"], w["n_kv_heads"]) == (12544, 66304, 98, 14)  # Table 6, 3.5x

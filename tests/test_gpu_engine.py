@@ -143,6 +143,19 @@ def test_streamed_7b_shape_step_matches_oracle():
         s.close()
 
 
+def test_streamed_long_context_chunked_step_matches_oracle():
+    """Two layers at 8192 tokens with the MLP in 2048-token chunks (K = 2, one segment: the forward keeps
+    both layers' internals, the attention half only, and the backward recomputes the MLP chunks): the
+    chunked path of the long-context workloads through the engine, against the oracle per tensor."""
+    shape = dict(hidden=896, n_q_heads=7, n_kv_heads=1, head_dim=128, ffn=2048)
+    s = Stack(shape, 2, 1, 8192, ckpt_interval=2, mlp_chunk=2048)
+    try:
+        y, dx, grads = s.step()
+        _check_against_oracle(s, y, dx, grads)
+    finally:
+        s.close()
+
+
 def _bit_exact_runs(shape, n_layers, B, T, K, variants):
     runs = {}
     for name, opts in variants.items():

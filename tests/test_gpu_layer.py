@@ -32,6 +32,9 @@ CASES = {
     # the Qwen2.5-14B layer shape
     "qwen14b_b1_t64": (dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824), 1, 64, 0),
     "qwen14b_b1_t1024": (dict(hidden=5120, n_q_heads=40, n_kv_heads=8, head_dim=128, ffn=13824), 1, 1024, 0),
+    # the long-context regime: 64 key blocks per query row on the tcgen05 attention, the MLP over four
+    # 2048-token chunks (the chunked path the 32K-token workload runs), a 7:1 head group
+    "gqa7_t8192_chunked": (dict(hidden=896, n_q_heads=7, n_kv_heads=1, head_dim=128, ffn=2048), 1, 8192, 2048),
 }
 
 

@@ -571,10 +571,10 @@ SWEEPS = {
     # pinned bf16 weights, beyond the host memory of the GPU machine next to the gradient slabs)
     "width": [dict(shape=width_shape(w), L=12, B=32, T=1024, K=4, chunk=0, label=f"width{w}x_x12")
               for w in (1.0, 1.5, 2.0, 2.5, 3.0, 3.5)],
-    # Table 7's longest rows: one sequence, MLP in 4096-token chunks (512K with the one-workspace schedule, whose
-    # per-layer internals of 21 GB would not fit K = 4 times next to the checkpoints)
-    "context": [dict(shape=QWEN7B, L=28, B=1, T=T, K=4, chunk=4096, label=f"7b_x28_b1x{T}",
-                     recompute_internals=int(T > 262144)) for T in (131072, 262144, 524288)],
+    # Table 7's longest rows: one sequence, MLP in 4096-token chunks (at 512K the four layer-internals sets take
+    # 83 GB and the whole workspace 167 GB of the B200's 192 GB)
+    "context": [dict(shape=QWEN7B, L=28, B=1, T=T, K=4, chunk=4096, label=f"7b_x28_b1x{T}")
+                for T in (131072, 262144, 524288)],
 }
 
 

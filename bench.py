@@ -310,21 +310,48 @@ def run_reference(args, cfg, rank, world):
 
 
 # ---------------------------------------------------------------- ours
-def fill_store(L_, store, cfg, n_layers, seed=1234):
+def fill_store(L_, store, cfg, n_layers, seed=1234, master=True):
+    """The synthetic weights of every layer: into the fp32 master and then the bf16 copy (RNE), or,
+    for a store without a master, one layer at a time through an fp32 scratch record."""
     off = L_.mt_layer_param_offsets(cfg)
     shapes = synth.layer_tensor_shapes(cfg.hidden, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn,
                                        bool(cfg.qkv_bias))
+    scratch = None if master else np.zeros(off.record_elems, dtype=np.float32)
     for l in range(n_layers):
-        ptr = L_.mt_host_store_master(store, l)
-        master = np.ctypeslib.as_array((ctypes.c_float * off.record_elems).from_address(ptr))
+        if master:
+            ptr = L_.mt_host_store_master(store, l)
+            rec = np.ctypeslib.as_array((ctypes.c_float * off.record_elems).from_address(ptr))
+        else:
+            rec = scratch
         for name, shp in shapes.items():
             o = getattr(off, name)
             n = int(np.prod(shp))
             if name in ("g1", "g2"):
-                master[o:o + n] = 1.0
+                rec[o:o + n] = 1.0
             else:
-                synth.normal_f32(seed, l, synth.TENSOR_IDS[name], n, synth.WEIGHT_STD, out=master[o:o + n])
-    L_.mt_host_store_refresh_bf16(store, 0)
+                synth.normal_f32(seed, l, synth.TENSOR_IDS[name], n, synth.WEIGHT_STD, out=rec[o:o + n])
+        if not master:
+            bf = np.ctypeslib.as_array((ctypes.c_uint16 * off.record_elems).from_address(L_.mt_host_store_bf16(store, l)))
+            bf[:] = synth.f32_to_bf16_bits(rec)
+    if master:
+        L_.mt_host_store_refresh_bf16(store, 0)
+
+
+def keep_master(L_, cfg, n_layers, args) -> bool:
+    """Whether this rank's host store can hold the fp32 master next to the bf16 copy: the optimizer sink
+    needs it; with the no-op sink it is kept whenever the host's available memory, shared by the ranks
+    of this node, holds every rank's store and slabs with 25% to spare."""
+    if args.sink == "adamw":
+        return True
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        return True
+    rec = L_.mt_layer_param_offsets(cfg).record_elems
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+    need = local * (n_layers * rec * 6 + 3 * rec * 4)
+    return 1.25 * need <= avail
 
 
 def run_ours(args, cfg, rank, world, local_rank):
@@ -346,8 +373,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     opts = L_.make_opts(ckpt_interval=abl.get("ckpt_interval", cfg["K"]), mlp_chunk=cfg["chunk"], time_gemms=1,
                         timeout_ms=120000, n_weight_slots=abl.get("n_weight_slots", 0),
                         no_slab_pool=abl.get("no_slab_pool", 0), recompute_internals=int(args.recompute_internals))
-    store = L_.mt_host_store_create(lcfg, nL, True)
-    fill_store(L_, store, lcfg, nL)
+    master = keep_master(L_, lcfg, nL, args)
+    store = L_.mt_host_store_create(lcfg, nL, master)
+    fill_store(L_, store, lcfg, nL, master=master)
     nbytes = L_.mt_engine_workspace_bytes(lcfg, nL, B, T, opts)
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     streams = [torch.cuda.Stream() for _ in range(3)]
@@ -506,7 +534,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                        "mlp_chunk": cfg["chunk"], "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each layer's weights alone are %.0f MB)" % (p_layer * 2 / 1e6),
                        "sink": ("CPU AdamW on the fp32 master + bf16 refresh (library sink)" if args.sink == "adamw"
-                                else "pinned slab handed to a no-op host callback")},
+                                else "pinned slab handed to a no-op host callback"),
+                       "host_store": ("pinned fp32 master + bf16 streaming copy" if master else
+                                      "pinned bf16 streaming copy only (the host's memory could not hold every "
+                                      "rank's fp32 master; the no-op sink does not read it)")},
             "tokens_per_s": B * T * world / (ms / 1e3),
             "clocks": clk,
             "e2e": {"value": e2e, "unit": UNIT,

@@ -432,3 +432,30 @@ def test_traced_step_gives_an_ordered_timeline():
         assert all(np.array_equal(g0[k], g1[k]) for k in g0)
     finally:
         s.close()
+
+
+def test_bench_store_fill_without_the_master_gives_the_same_bf16_record():
+    """bench.py fills a host store without an fp32 master (when the host's memory cannot hold every rank's)
+    one record at a time through an fp32 scratch; the bf16 copy streamed to the GPU is bitwise the one the
+    master-plus-refresh path gives."""
+    import importlib.util
+    import os
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(os.path.dirname(os.path.dirname(
+        os.path.abspath(__file__))), "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    cfg = L.make_cfg(**TINY)
+    rec = L.mt_layer_param_offsets(cfg).record_elems
+    a = L.mt_host_store_create(cfg, 2, True)
+    b = L.mt_host_store_create(cfg, 2, False)
+    try:
+        bench.fill_store(L, a, cfg, 2, master=True)
+        bench.fill_store(L, b, cfg, 2, master=False)
+        assert L.mt_host_store_master(b, 0) is None or L.mt_host_store_master(b, 0) == 0
+        for l in range(2):
+            ba = np.ctypeslib.as_array((ctypes.c_uint16 * rec).from_address(L.mt_host_store_bf16(a, l)))
+            bb = np.ctypeslib.as_array((ctypes.c_uint16 * rec).from_address(L.mt_host_store_bf16(b, l)))
+            assert np.array_equal(ba, bb), l
+    finally:
+        L.mt_host_store_destroy(a)
+        L.mt_host_store_destroy(b)

@@ -316,3 +316,18 @@ def test_sweep_points_fit_the_device_and_the_host():
         assert n1 - n0 == ((l1 + 3) // 4 - (l0 + 3) // 4) * act
     w = bench.width_shape(3.5)
     assert (w["hidden"], w["ffn"], w["n_q_heads"], w["n_kv_heads"]) == (12544, 66304, 98, 14)  # Table 6, 3.5x
+
+
+def test_bench_keeps_the_fp32_master_unless_the_host_cannot_hold_it(monkeypatch):
+    import importlib.util
+    import types
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    cfg = L.make_cfg(**QWEN7B)
+    args = types.SimpleNamespace(sink="none")
+    monkeypatch.setenv("LOCAL_WORLD_SIZE", "1")
+    assert bench.keep_master(L, cfg, 1, args)  # one 7B layer: 1.4 GB
+    monkeypatch.setenv("LOCAL_WORLD_SIZE", "100000")
+    assert not bench.keep_master(L, cfg, 28, args)  # far beyond any host
+    assert bench.keep_master(L, cfg, 28, types.SimpleNamespace(sink="adamw"))  # the optimizer needs it

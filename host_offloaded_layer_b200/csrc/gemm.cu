@@ -112,6 +112,15 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
   return __fdividef(1.0f, 1.0f + e);
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (a hint: nothing is written). The
+// caller keeps the range inside one buffer it reads later; a start that is not
+// 16-byte aligned is skipped and the size is rounded down to 16 bytes.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  bytes &= ~15u;
+  if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0 || bytes == 0) return;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Epilogue of one 32-column chunk of one output row.
 __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0, const uint32_t (&r)[32]) {
   float v[32];
@@ -608,12 +617,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;          // TMEM lanes [32 q, 32 q + 32)
     const int hc = (warp - 2) >> 2;  // N-half of the accumulator this warp drains
+    // The epilogues that read global memory (g and u of the SwiGLU backward, the
+    // residual, the dot operand) read one row per thread, 64 bytes at a time: from
+    // DRAM that is latency-bound. Each thread therefore prefetches its row's span
+    // of a tile into L2 one tile ahead, while the tile before it drains (with two
+    // accumulators only: with one, the next tile is a whole main loop away).
+    auto prefetch_rows = [&](int t) {
+      if (NACC != 2 || t >= num_tiles || ep.swiglu == 1 || ep.rope_tab) return;
+      if (ep.swiglu != 2 && !ep.res && !ep.dot_with) return;
+      int mb, nb;
+      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
+      const int col0 = nb * BN + hc * 256;
+      const int ncol = min(256, ep.N - col0);
+      if (row >= ep.M || ncol <= 0) return;
+      const uint32_t bytes = static_cast<uint32_t>(ncol) * 2u;
+      if (ep.swiglu == 2) {
+        const __nv_bfloat16* g = ep.gu + static_cast<int64_t>(row) * ep.ld_gu + col0;
+        prefetch_l2(g, bytes);
+        prefetch_l2(g + ep.F, bytes);
+      } else {
+        if (ep.res) prefetch_l2(ep.res + static_cast<int64_t>(row) * ep.ldr + col0, bytes);
+        if (ep.dot_with) prefetch_l2(ep.dot_with + static_cast<int64_t>(row) * ep.ld_dot + col0, bytes);
+      }
+    };
+    prefetch_rows(cluster);
     int tl = 0;
     for (int t = cluster; t < num_tiles; t += n_clusters, ++tl) {
       const int ab = NACC == 2 ? (tl & 1) : 0;
       const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
       int mb, nb;
       tile_coords(t, num_m, num_n, ep.raster, mb, nb);
+      prefetch_rows(t + n_clusters);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
@@ -777,10 +812,22 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
 // layout with K >= 8192, and any plain epilogue with K >= 8192 and M >= 65536.
 // Every other launch runs the 256 x 256 tile with three stages of 128-wide K
 // (eight MMAs per barrier round trip measured 7-16% faster than four).
+// A launch whose wide tiles leave a last round of clusters mostly idle (the
+// 3584 x 3584 weight gradient: 98 tiles of 256 x 512 on 74 clusters, two rounds,
+// against 196 of 256 x 256 in three) runs the 256 x 256 tile: the wide tile is
+// taken only while its rounds of clusters, each costing about 1.8 narrow rounds
+// (it is 4-13% faster per FLOP), are not more than the narrow tile's.
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
   const bool plain = ep.swiglu == 0 && !ep.rope_tab && !ep.dot_with;
-  const bool wide = plain && ep.K >= 8192 && ((A_MN && B_MN) || ep.M >= 65536);
+  bool wide = plain && ep.K >= 8192 && ((A_MN && B_MN) || ep.M >= 65536);
+  if (wide) {
+    const int64_t num_m = (ep.M + c2::BM - 1) / c2::BM;
+    const int64_t clusters = std::max(1, max_pair_clusters<A_MN, B_MN, 1, 2>());
+    const int64_t rounds_wide = (num_m * ((ep.N + 511) / 512) + clusters - 1) / clusters;
+    const int64_t rounds_narrow = (num_m * ((ep.N + 255) / 256) + clusters - 1) / clusters;
+    wide = 18 * rounds_wide <= 10 * rounds_narrow;
+  }
   if (wide) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
   return launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st);
 }

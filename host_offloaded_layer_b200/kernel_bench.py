@@ -1,6 +1,7 @@
 """Times one block kernel through the C ABI (CUDA events, warm-up first).
 
     python -m host_offloaded_layer_b200.kernel_bench gemm --M 16384 --N 4608 --K 3584 --layout kk
+    python -m host_offloaded_layer_b200.kernel_bench gemm --M 98304 --N 3584 --K 3584 --layout kk --res
     python -m host_offloaded_layer_b200.kernel_bench gemm_swiglu --M 8192 --F 18944 --K 3584
     python -m host_offloaded_layer_b200.kernel_bench gemm_swiglu_bwd --M 8192 --F 18944 --K 3584
     python -m host_offloaded_layer_b200.kernel_bench attn_fwd --B 8 --T 1024 --nq 28 --nkv 4 --d 128
@@ -41,6 +42,7 @@ def main():
     ap.add_argument("--K", type=int, default=3584)
     ap.add_argument("--layout", default="kk", choices=["kk", "km", "mk", "mm"])
     ap.add_argument("--f32", action="store_true", help="fp32 output (weight-gradient epilogue)")
+    ap.add_argument("--res", action="store_true", help="add a bf16 residual (the O / down projection epilogue)")
     ap.add_argument("--B", type=int, default=8)
     ap.add_argument("--T", type=int, default=1024)
     ap.add_argument("--nq", type=int, default=28)
@@ -63,10 +65,11 @@ def main():
         C = torch.empty(a.M * a.N, dtype=torch.float32 if a.f32 else torch.bfloat16, device="cuda")
         lda = a.M if a_mn else a.K
         ldb = a.N if b_mn else a.K
+        R = _dev(torch, a.M * a.N, 3) if a.res else None
         fn = lambda: L.mt_gemm_bf16(A, lda, int(a_mn), B, ldb, int(b_mn), C, a.N, int(a.f32), 0, a.M, a.N, a.K,  # noqa
-                                    stream=st)
+                                    None, R, a.N if a.res else 0, stream=st)
         work, unit = 2.0 * a.M * a.N * a.K, "TFLOP/s"
-        shape = dict(M=a.M, N=a.N, K=a.K, layout=a.layout, f32=a.f32)
+        shape = dict(M=a.M, N=a.N, K=a.K, layout=a.layout, f32=a.f32, res=a.res)
     elif a.op == "gemm_swiglu":
         # the gate/up projection with the SwiGLU epilogue (m, and g and u for the backward)
         A = _dev(torch, a.M * a.K, 1)

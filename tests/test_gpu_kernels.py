@@ -26,7 +26,7 @@ def _check_dev_error():
 # ------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 300, 136), (2048, 4096, 512), (96, 40, 1000),
-                                   (600, 1100, 8200)])  # K >= 8192: the 256 x 512 tile on the MN / MN layout
+                                   (600, 1100, 8200)])  # K >= 8192, a few tiles: the 256 x 256 tile
 def test_gemm_layouts_match_fp64_matmul(a_mn, b_mn, M, N, K):
     import torch
     lda = ((M if a_mn else K) + 7) // 8 * 8 + 8
@@ -81,13 +81,37 @@ def test_gemm_is_deterministic_and_covers_many_waves():
     _check_dev_error()
 
 
+def test_gemm_weight_gradient_layout_wide_tile():
+    """The weight-gradient layout (both operands MN-major) with K >= 8192 runs the 256 x 512 pair
+    tile when its rounds of clusters pay: 2000 x 4000 is 64 wide tiles (one round) against 128
+    narrow ones (two). fp32 output, then fp32 accumulate, on sampled rows against float64, with
+    ragged row and column blocks."""
+    import torch
+    M, N, K = 2000, 4000, 8200
+    A = _bits(14, 1, K * M).reshape(K, M)  # [K, M]: M contiguous
+    B = _bits(14, 2, K * N, 0.05).reshape(K, N)
+    dA, dB = H.dev_bf16(A), H.dev_bf16(B)
+    C = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    L.mt_gemm_bf16(dA, M, 1, dB, N, 1, C, N, 1, 0, M, N, K)
+    torch.cuda.synchronize()
+    _check_dev_error()
+    rows = np.concatenate([np.random.default_rng(4).choice(M - 16, 48, replace=False), np.arange(M - 16, M)])
+    ref = H.bits_to_f64(A[:, rows]).T @ H.bits_to_f64(B)
+    assert H.rel(H.host_f64(C)[rows], ref) < 1e-5
+    L.mt_gemm_bf16(dA, M, 1, dB, N, 1, C, N, 1, 1, M, N, K)
+    torch.cuda.synchronize()
+    assert H.rel(H.host_f64(C)[rows], 2 * ref) < 1e-5
+    _check_dev_error()
+
+
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1)])
 def test_gemm_long_k_many_rows_wide_tile(a_mn, b_mn):
     """At 65536 rows and more with K >= 8192 the forward and input-gradient layouts run the
     256 x 512 pair tile (the down projection and dh2 of the 96 x 1024 workload): sampled rows
-    of a bf16 result with a residual against the float64 product, and a ragged last row block."""
+    of a bf16 result with a residual against the float64 product, a ragged last row block and a
+    ragged last column block (N = 1000: 514 wide tiles, whole rounds of 64 to 74 clusters)."""
     import torch
-    M, N, K = 65600, 384, 8200
+    M, N, K = 65600, 1000, 8200
     A = _bits(13, 1, M * K).reshape(M, K)
     b_rows, b_cols = (K, N) if b_mn else (N, K)
     B = _bits(13, 2, b_rows * b_cols, 0.05).reshape(b_rows, b_cols)

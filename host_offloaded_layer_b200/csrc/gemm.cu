@@ -112,15 +112,6 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
   return __fdividef(1.0f, 1.0f + e);
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (a hint: nothing is written). The
-// caller keeps the range inside one buffer it reads later; a start that is not
-// 16-byte aligned is skipped and the size is rounded down to 16 bytes.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  bytes &= ~15u;
-  if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0 || bytes == 0) return;
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // Epilogue of one 32-column chunk of one output row.
 __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0, const uint32_t (&r)[32]) {
   float v[32];
@@ -451,6 +442,11 @@ __device__ __forceinline__ uint32_t rows_bytes(bool mn, int r0, int R) {
   return b;
 }
 
+// TMA warp, MMA warp and four epilogue warps per 256 accumulator columns, one
+// per TMEM lane quarter. Measured and not kept: eight epilogue warps on the
+// 256 x 256 tile (5-12% slower on every shape of the layer), an L2 prefetch of
+// the next tile's epilogue operands and register double-buffering of the
+// SwiGLU backward's g / u loads (no gain; 15% slower).
 constexpr int threads2(int nh) { return 64 + 128 * nh; }
 
 // KA: 64-wide K atoms per pipeline stage (NH = 1: 1 -> 6 stages of 64, 2 -> 3
@@ -617,38 +613,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads2(NH), 1)
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;          // TMEM lanes [32 q, 32 q + 32)
     const int hc = (warp - 2) >> 2;  // N-half of the accumulator this warp drains
-    // The epilogues that read global memory (g and u of the SwiGLU backward, the
-    // residual, the dot operand) read one row per thread, 64 bytes at a time: from
-    // DRAM that is latency-bound. Each thread therefore prefetches its row's span
-    // of a tile into L2 one tile ahead, while the tile before it drains (with two
-    // accumulators only: with one, the next tile is a whole main loop away).
-    auto prefetch_rows = [&](int t) {
-      if (NACC != 2 || t >= num_tiles || ep.swiglu == 1 || ep.rope_tab) return;
-      if (ep.swiglu != 2 && !ep.res && !ep.dot_with) return;
-      int mb, nb;
-      tile_coords(t, num_m, num_n, ep.raster, mb, nb);
-      const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;
-      const int col0 = nb * BN + hc * 256;
-      const int ncol = min(256, ep.N - col0);
-      if (row >= ep.M || ncol <= 0) return;
-      const uint32_t bytes = static_cast<uint32_t>(ncol) * 2u;
-      if (ep.swiglu == 2) {
-        const __nv_bfloat16* g = ep.gu + static_cast<int64_t>(row) * ep.ld_gu + col0;
-        prefetch_l2(g, bytes);
-        prefetch_l2(g + ep.F, bytes);
-      } else {
-        if (ep.res) prefetch_l2(ep.res + static_cast<int64_t>(row) * ep.ldr + col0, bytes);
-        if (ep.dot_with) prefetch_l2(ep.dot_with + static_cast<int64_t>(row) * ep.ld_dot + col0, bytes);
-      }
-    };
-    prefetch_rows(cluster);
     int tl = 0;
     for (int t = cluster; t < num_tiles; t += n_clusters, ++tl) {
       const int ab = NACC == 2 ? (tl & 1) : 0;
       const uint32_t aph = static_cast<uint32_t>(NACC == 2 ? (tl >> 1) : tl) & 1u;
       int mb, nb;
       tile_coords(t, num_m, num_n, ep.raster, mb, nb);
-      prefetch_rows(t + n_clusters);
       if (!warp_wait(smem_u32(&tfull[ab]), aph, abort_flag, err, DEV_ERR_TIMEOUT_EPILOGUE)) break;
       fence_after();
       const int row = mb * BM + static_cast<int>(rank) * 128 + q * 32 + lane;

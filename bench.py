@@ -522,7 +522,8 @@ def run_ours(args, cfg, rank, world, local_rank):
 
         t_comp = st.exec_flops / (peak_tf * 1e12)
         t_roof = t_roof_at(peak_tf)
-        cpu_tf, cpu_desc, cpu_threads, cpu_sec, cpu_T = oracle_sample(cfg, budget_s=12.0)
+        if world == 1:  # the CPU baseline is timed at one GPU only
+            cpu_tf, cpu_desc, cpu_threads, cpu_sec, cpu_T = oracle_sample(cfg, budget_s=12.0)
         tr = st_tr.trace
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -567,12 +568,12 @@ def run_ours(args, cfg, rank, world, local_rank):
                          "step_ms": tr.span_ms, "fwd_ms": tr.fwd_ms, "refwd_ms": tr.refwd_ms, "bwd_ms": tr.bwd_ms,
                          "h2d_ms": tr.h2d_ms, "d2h_ms": tr.d2h_ms, "exposed_h2d_ms": tr.exposed_h2d_ms,
                          "exposed_d2h_ms": tr.exposed_d2h_ms, "idle_other_ms": tr.idle_other_ms},
-            "cpu_baseline": {"value": cpu_tf, "unit": UNIT, "cores": cpu_threads, "kind": "oracle",
-                             "sample": cpu_desc,
-                             "step_s_extrapolated": oracle_step_extrapolated(cfg, p_layer, cpu_sec, cpu_T),
-                             "extrapolation": ("the oracle's forward+backward of every layer on all B x T tokens "
-                                               "(no recompute), scaled from the sample: projections linearly in "
-                                               "tokens, attention in B x T^2 (extrapolated, not measured)")},
+            "cpu_baseline": None if world > 1 else {
+                "value": cpu_tf, "unit": UNIT, "cores": cpu_threads, "kind": "oracle", "sample": cpu_desc,
+                "step_s_extrapolated": oracle_step_extrapolated(cfg, p_layer, cpu_sec, cpu_T),
+                "extrapolation": ("the oracle's forward+backward of every layer on all B x T tokens "
+                                  "(no recompute), scaled from the sample: projections linearly in "
+                                  "tokens, attention in B x T^2 (extrapolated, not measured)")},
             "device_workspace_gb": nbytes / 1e9,
         }
     L_.mt_engine_destroy(eng)

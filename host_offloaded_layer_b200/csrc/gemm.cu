@@ -75,6 +75,9 @@ struct EpiArgs {
   int64_t ld_dot;
   float* dot_out;
   int dot_hd, dot_T, dot_heads;
+  // 32-byte row chunks (base and row stride multiples of 32 bytes): the epilogue
+  // moves C, the residual and g / u with 256-bit accesses, one whole sector each
+  int c_v8, res_v8, gu_v8;
 };
 
 // Output-tile order. raster 0: groups of 16 row-blocks, columns within a
@@ -103,6 +106,11 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
+__device__ __forceinline__ uint32_t pack_bf16_pair(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with the MUFU ex2 and a fast divide
 // (relative error well below bf16 rounding; 2^x saturates to 0 / inf, giving
 // sigmoid 1 / 0 at the extremes).
@@ -110,6 +118,32 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
   float e;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z));
   return __fdividef(1.0f, 1.0f + e);
+}
+
+// 256-bit global accesses (32 bytes, one L2 sector; p 32-byte aligned). A row
+// per thread reads and writes 64 or 128 bytes per 32-column chunk: 16-byte
+// accesses would touch each sector twice.
+__device__ __forceinline__ void ld_v8(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p)
+               : "memory");
+}
+__device__ __forceinline__ void ld_v8_cs(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p)
+               : "memory");
+}
+__device__ __forceinline__ void st_v8(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]),
+               "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void st_v8_cs(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]),
+               "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 // Epilogue of one 32-column chunk of one output row.
@@ -130,16 +164,55 @@ __device__ __forceinline__ void store_chunk(const EpiArgs& ep, int row, int col0
       }
     }
     if (ep.res) {
-      const uint4* rp = reinterpret_cast<const uint4*>(ep.res + static_cast<int64_t>(row) * ep.ldr + col0);
+      const __nv_bfloat16* rrow = ep.res + static_cast<int64_t>(row) * ep.ldr + col0;
+      if (ep.res_v8) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 u = rp[q];
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t w[8];
+          ld_v8(rrow + hh * 16, w);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[q * 8 + j] += bf2f(h[j]);
+          for (int j = 0; j < 8; ++j) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+            v[hh * 16 + 2 * j] += f.x;
+            v[hh * 16 + 2 * j + 1] += f.y;
+          }
+        }
+      } else {
+        const uint4* rp = reinterpret_cast<const uint4*>(rrow);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 u = rp[q];
+          const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[q * 8 + j] += bf2f(h[j]);
+        }
       }
     }
-    if (ep.c_f32) {
+    if (ep.c_f32 && ep.c_v8) {
+      float* cp = static_cast<float*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        uint32_t w[8];
+        if (ep.accumulate) {
+          ld_v8(cp + hh * 8, w);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[j] = __float_as_uint(__uint_as_float(w[j]) + v[hh * 8 + j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[j] = __float_as_uint(v[hh * 8 + j]);
+        }
+        st_v8(cp + hh * 8, w);
+      }
+    } else if (!ep.c_f32 && ep.c_v8) {
+      __nv_bfloat16* cp = static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = pack_bf16_pair(v[hh * 16 + 2 * j], v[hh * 16 + 2 * j + 1]);
+        st_v8(cp + hh * 16, w);
+      }
+    } else if (ep.c_f32) {
       float4* cp = reinterpret_cast<float4*>(static_cast<float*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -263,7 +336,28 @@ __device__ __forceinline__ float store_chunk_dot(const EpiArgs& ep, int row, int
 // g and u in place (each element is read and written by the same thread).
 __device__ __forceinline__ void store_swiglu_bwd(const EpiArgs& ep, int row, int f0, const uint32_t (&r)[32]) {
   __nv_bfloat16* grow = ep.gu + static_cast<int64_t>(row) * ep.ld_gu;
-  if (f0 + 32 <= ep.F) {
+  if (f0 + 32 <= ep.F && ep.gu_v8) {
+    uint32_t gw[2][8], uw[2][8];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      ld_v8_cs(grow + f0 + hh * 16, gw[hh]);
+      ld_v8_cs(grow + ep.F + f0 + hh * 16, uw[hh]);
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[hh][j]));
+        const float2 u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[hh][j]));
+        const float d0 = __uint_as_float(r[hh * 16 + 2 * j]), d1 = __uint_as_float(r[hh * 16 + 2 * j + 1]);
+        const float s0 = sigmoid_fast(g.x), s1 = sigmoid_fast(g.y);
+        gw[hh][j] = pack_bf16_pair(d0 * u.x * s0 * (1.0f + g.x * (1.0f - s0)), d1 * u.y * s1 * (1.0f + g.y * (1.0f - s1)));
+        uw[hh][j] = pack_bf16_pair(d0 * g.x * s0, d1 * g.y * s1);
+      }
+      st_v8_cs(grow + f0 + hh * 16, gw[hh]);
+      st_v8_cs(grow + ep.F + f0 + hh * 16, uw[hh]);
+    }
+  } else if (f0 + 32 <= ep.F) {
     uint4* gp = reinterpret_cast<uint4*>(grow + f0);
     uint4* up = reinterpret_cast<uint4*>(grow + ep.F + f0);
     // g and u are read once and written once: streaming loads / stores keep them from
@@ -318,7 +412,24 @@ __device__ __forceinline__ void store_swiglu(const EpiArgs& ep, int row, int f0,
   }
   __nv_bfloat16* mrow = static_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc;
   __nv_bfloat16* grow = ep.gu ? ep.gu + static_cast<int64_t>(row) * ep.ld_gu : nullptr;
-  if (f0 + 32 <= ep.F) {
+  if (f0 + 32 <= ep.F && ep.c_v8 && (!grow || ep.gu_v8)) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t wm[8], wg[8], wu[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = hh * 16 + 2 * j;
+        wm[j] = pack_bf16_pair(m[e], m[e + 1]);
+        wg[j] = pack_bf16_pair(__uint_as_float(rg[e]), __uint_as_float(rg[e + 1]));
+        wu[j] = pack_bf16_pair(__uint_as_float(ru[e]), __uint_as_float(ru[e + 1]));
+      }
+      st_v8(mrow + f0 + hh * 16, wm);
+      if (grow) {
+        st_v8(grow + f0 + hh * 16, wg);
+        st_v8(grow + ep.F + f0 + hh * 16, wu);
+      }
+    }
+  } else if (f0 + 32 <= ep.F) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 um, ug, uu;
@@ -788,7 +899,13 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
 // taken only while its rounds of clusters, each costing about 1.8 narrow rounds
 // (it is 4-13% faster per FLOP), are not more than the narrow tile's.
 template <bool A_MN, bool B_MN>
-mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, const EpiArgs& ep, cudaStream_t st) {
+mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, EpiArgs ep, cudaStream_t st) {
+  // 256-bit epilogue accesses where every 32-column row chunk is 32-byte aligned: the base pointer and
+  // the row stride in bytes are multiples of 32 (chunks start every 32 columns)
+  auto a32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };
+  ep.c_v8 = ep.C && a32(ep.C) && (ep.ldc * (ep.c_f32 ? 4 : 2)) % 32 == 0;
+  ep.res_v8 = ep.res && a32(ep.res) && (ep.ldr * 2) % 32 == 0;
+  ep.gu_v8 = ep.gu && a32(ep.gu) && (ep.ld_gu * 2) % 32 == 0 && (static_cast<int64_t>(ep.F) * 2) % 32 == 0;
   const bool plain = ep.swiglu == 0 && !ep.rope_tab && !ep.dot_with;
   bool wide = plain && ep.K >= 8192 && ((A_MN && B_MN) || ep.M >= 65536);
   if (wide) {
@@ -864,6 +981,7 @@ EpiArgs plain_epilogue(int64_t M, int64_t N, int64_t K) {
   ep.F = 0;
   ep.gu = nullptr;
   ep.ld_gu = 0;
+  ep.c_v8 = ep.res_v8 = ep.gu_v8 = 0;
   ep.rope_tab = nullptr;
   ep.rope_cols = ep.rope_hd = ep.rope_T = 0;
   ep.dot_with = nullptr;

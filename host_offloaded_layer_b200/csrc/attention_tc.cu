@@ -126,7 +126,8 @@ __device__ __forceinline__ FwdTile fwd_tile(int t, int n_qb, int nq, int B) {
 
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16* __restrict__ o, int64_t ld_o,
-                       float* __restrict__ lse, int B, int T, int nq, int nkv, float scale_log2, int32_t* err) {
+                       int o_v8, float* __restrict__ lse, int B, int T, int nq, int nkv, float scale_log2,
+                       int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
@@ -423,7 +424,22 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         uint32_t u0[32], u1[32];
         tmem_ld32(tmem + lane_base + COL_O + oc, u0);
         tmem_ld32(tmem + lane_base + COL_O + D + oc, u1);
-        if (q_row < T) {
+        if (q_row < T && o_v8) {
+          // whole 32-byte sectors: two 256-bit stores of 16 columns
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c0 = hh * 16 + 2 * e;
+              w[e] = pack_bf16((__uint_as_float(u0[c0]) * f0 + __uint_as_float(u1[c0]) * f1) * inv,
+                               (__uint_as_float(u0[c0 + 1]) * f0 + __uint_as_float(u1[c0 + 1]) * f1) * inv);
+            }
+            asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(orow + oc + hh * 16), "r"(w[0]),
+                         "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                         : "memory");
+          }
+        } else if (q_row < T) {
 #pragma unroll
           for (int qd = 0; qd < 4; ++qd) {
             float v[8];
@@ -473,8 +489,10 @@ mt_status attn_fwd_tc_launch(const mt_bf16* qkv, int64_t ld, mt_bf16* o, int64_t
   if (n_tiles >= (1ll << 31)) return fail(MT_ERR_INVALID_ARG, "attention: too many tiles");
   const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
   const float scale_log2 = LOG2E / sqrtf(static_cast<float>(D));
-  attn_fwd_tc_kernel<<<grid, FWD_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, lse, B, T,
-                                                            nq, nkv, scale_log2, err);
+  // 256-bit stores of O when every row's 32-column chunk is 32-byte aligned
+  const int o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 && (ld_o * 2) % 32 == 0;
+  attn_fwd_tc_kernel<<<grid, FWD_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<__nv_bfloat16*>(o), ld_o, o_v8, lse,
+                                                            B, T, nq, nkv, scale_log2, err);
   MT_TRY(launch_check("attn_fwd_tc_kernel"));
   add_exec_flops(4.0 * B * nq * D * (0.5 * double(T) * double(T)));
   return MT_OK;

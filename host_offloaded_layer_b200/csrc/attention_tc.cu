@@ -94,6 +94,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One 256-bit store (16 bf16 values, a whole 32-byte sector); p 32-byte aligned.
+__device__ __forceinline__ void st_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // The k-th tile of this CTA in a persistent walk over tiles sorted longest first: round k hands
 // out tiles [k G, k G + G) to the G CTAs in alternating directions (a snake), so the CTA that
 // takes the longest tile of one round takes the shortest of the next and the work stays even.
@@ -537,8 +544,8 @@ constexpr int BWD_THREADS = 64 + 256;
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
                            const __grid_constant__ CUtensorMap tm_do64, const float* __restrict__ lse,
-                           const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int T,
-                           int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
+                           const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int v8,
+                           int T, int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
                            int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -777,12 +784,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               pa[q] = pack_bf16(a0 * cs.x + b0 * cs.y, a1 * cs.z + b1 * cs.w);
               pb[q] = pack_bf16(b0 * cs.x - a0 * cs.y, b1 * cs.z - a1 * cs.w);
             }
+            if (v8) {
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              *reinterpret_cast<uint4*>(out + cp * 32 + qd * 8) =
-                  make_uint4(pa[4 * qd], pa[4 * qd + 1], pa[4 * qd + 2], pa[4 * qd + 3]);
-              *reinterpret_cast<uint4*>(out + (cp + 2) * 32 + qd * 8) =
-                  make_uint4(pb[4 * qd], pb[4 * qd + 1], pb[4 * qd + 2], pb[4 * qd + 3]);
+              for (int hh = 0; hh < 2; ++hh) {
+                st_v8(out + cp * 32 + hh * 16, pa + 8 * hh);
+                st_v8(out + (cp + 2) * 32 + hh * 16, pb + 8 * hh);
+              }
+            } else {
+#pragma unroll
+              for (int qd = 0; qd < 4; ++qd) {
+                *reinterpret_cast<uint4*>(out + cp * 32 + qd * 8) =
+                    make_uint4(pa[4 * qd], pa[4 * qd + 1], pa[4 * qd + 2], pa[4 * qd + 3]);
+                *reinterpret_cast<uint4*>(out + (cp + 2) * 32 + qd * 8) =
+                    make_uint4(pb[4 * qd], pb[4 * qd + 1], pb[4 * qd + 2], pb[4 * qd + 3]);
+              }
             }
           }
         }
@@ -795,7 +810,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t u[32];
           tmem_ld32(tmem + lane_base + col + ch * 32, u);
-          if (kv_row < T) {
+          if (kv_row < T && v8) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]) * f, __uint_as_float(u[2 * e + 1]) * f);
+            st_v8(out + ch * 32, w);
+            st_v8(out + ch * 32 + 16, w + 8);
+          } else if (kv_row < T) {
 #pragma unroll
             for (int qd = 0; qd < 4; ++qd) {
               uint4 w;
@@ -835,8 +856,8 @@ constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
                           const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
-                          const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int B, int T,
-                          int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
+                          const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, int64_t ld, int v8, int B,
+                          int T, int nq, int nkv, float scale_log2, float scale, const float2* __restrict__ rope,
                           int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1088,7 +1109,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             }
           }
         }
-        if (q_row < T) {
+        if (q_row < T && v8) {
+          uint32_t wv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            wv[e] = pack_bf16(__uint_as_float(u[2 * e]) * scale, __uint_as_float(u[2 * e + 1]) * scale);
+          st_v8(out + ch * 32, wv);
+          st_v8(out + ch * 32 + 16, wv + 8);
+        } else if (q_row < T) {
 #pragma unroll
           for (int qd = 0; qd < 4; ++qd) {
             uint4 wv;
@@ -1146,12 +1174,14 @@ mt_status attn_bwd_tc_launch(const mt_bf16* qkv, int64_t ld, const mt_bf16* d_o,
   const int64_t dq_tiles = static_cast<int64_t>((T + 127) / 128) * nq * B;
   const int gq = static_cast<int>(std::min<int64_t>(dq_tiles, num_sms()));
   const float2* rope = reinterpret_cast<const float2*>(rope_tab);
-  attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, B, T, nq, nkv,
-                                                                scale_log2, scale, rope, err);
+  // 256-bit stores of dq, dk, dv when every row's 32-column chunk is 32-byte aligned
+  const int v8 = (reinterpret_cast<uintptr_t>(dqkv) & 31u) == 0 && (ld * 2) % 32 == 0;
+  attn_bwd_dq_tc_kernel<<<gq, BWD_THREADS, DQ_SMEM_BYTES, st>>>(qkv128, do128, qkv64, lse, delta, out, ld, v8, B, T, nq,
+                                                                nkv, scale_log2, scale, rope, err);
   MT_TRY(launch_check("attn_bwd_dq_tc_kernel"));
   dim3 gk(nkv, B, (T + 127) / 128);
-  attn_bwd_dkv_tc_kernel<<<gk, BWD_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, T, nq, nkv,
-                                                                 scale_log2, scale, rope, err);
+  attn_bwd_dkv_tc_kernel<<<gk, BWD_THREADS, KV_SMEM_BYTES, st>>>(qkv128, qkv64, do64, lse, delta, out, ld, v8, T, nq,
+                                                                 nkv, scale_log2, scale, rope, err);
   MT_TRY(launch_check("attn_bwd_dkv_tc_kernel"));
   // dq: QK^T, dO V^T, dS K; dkv: QK^T, dO V^T, P^T dO, dS^T Q (causal half)
   add_exec_flops(14.0 * B * nq * D * (0.5 * double(T) * double(T)));

@@ -893,10 +893,10 @@ mt_status launch_2sm_ka(const CUtensorMap& ta, const CUtensorMap& tb, const EpiA
 // layout with K >= 8192, and any plain epilogue with K >= 8192 and M >= 65536.
 // Every other launch runs the 256 x 256 tile with three stages of 128-wide K
 // (eight MMAs per barrier round trip measured 7-16% faster than four).
-// A launch whose wide tiles leave a last round of clusters mostly idle (the
-// 3584 x 3584 weight gradient: 98 tiles of 256 x 512 on 74 clusters, two rounds,
+// A launch whose wide tiles leave a last wave of clusters mostly idle (the
+// 3584 x 3584 weight gradient: 98 tiles of 256 x 512 on 74 clusters, two waves,
 // against 196 of 256 x 256 in three) runs the 256 x 256 tile: the wide tile is
-// taken only while its rounds of clusters, each costing about 1.8 narrow rounds
+// taken only while its waves of clusters, each costing about 1.8 narrow waves
 // (it is 4-13% faster per FLOP), are not more than the narrow tile's.
 template <bool A_MN, bool B_MN>
 mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, EpiArgs ep, cudaStream_t st) {
@@ -911,9 +911,9 @@ mt_status launch_2sm(const CUtensorMap& ta, const CUtensorMap& tb, EpiArgs ep, c
   if (wide) {
     const int64_t num_m = (ep.M + c2::BM - 1) / c2::BM;
     const int64_t clusters = std::max(1, max_pair_clusters<A_MN, B_MN, 1, 2>());
-    const int64_t rounds_wide = (num_m * ((ep.N + 511) / 512) + clusters - 1) / clusters;
-    const int64_t rounds_narrow = (num_m * ((ep.N + 255) / 256) + clusters - 1) / clusters;
-    wide = 18 * rounds_wide <= 10 * rounds_narrow;
+    const int64_t waves_wide = (num_m * ((ep.N + 511) / 512) + clusters - 1) / clusters;
+    const int64_t waves_narrow = (num_m * ((ep.N + 255) / 256) + clusters - 1) / clusters;
+    wide = 18 * waves_wide <= 10 * waves_narrow;
   }
   if (wide) return launch_2sm_ka<A_MN, B_MN, 1, 2>(ta, tb, ep, st);
   return launch_2sm_ka<A_MN, B_MN, 2, 1>(ta, tb, ep, st);

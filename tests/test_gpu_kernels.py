@@ -83,7 +83,7 @@ def test_gemm_is_deterministic_and_covers_many_waves():
 
 def test_gemm_weight_gradient_layout_wide_tile():
     """The weight-gradient layout (both operands MN-major) with K >= 8192 runs the 256 x 512 pair
-    tile when its rounds of clusters pay: 2000 x 4000 is 64 wide tiles (one round) against 128
+    tile when its waves of clusters pay: 2000 x 4000 is 64 wide tiles (one wave) against 128
     narrow ones (two). fp32 output, then fp32 accumulate, on sampled rows against float64, with
     ragged row and column blocks."""
     import torch
@@ -109,7 +109,7 @@ def test_gemm_long_k_many_rows_wide_tile(a_mn, b_mn):
     """At 65536 rows and more with K >= 8192 the forward and input-gradient layouts run the
     256 x 512 pair tile (the down projection and dh2 of the 96 x 1024 workload): sampled rows
     of a bf16 result with a residual against the float64 product, a ragged last row block and a
-    ragged last column block (N = 1000: 514 wide tiles, whole rounds of 64 to 74 clusters)."""
+    ragged last column block (N = 1000: 514 wide tiles, whole waves of 64 to 74 clusters)."""
     import torch
     M, N, K = 65600, 1000, 8200
     A = _bits(13, 1, M * K).reshape(M, K)
